@@ -1,0 +1,526 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA2 decode step on B200.
+
+One step = one decode step of an 8-layer CSA2 stack (Full, Reindex, Reindex, Reuse x 5) for a batch
+of sequences: quantize-append of the new entry, the Full-mode indexer over every cached entry, two
+Reindex-mode indexers over the pool, and sparse attention in every layer. Default workload: B = 8
+sequences of N = 1,048,576 entries (the million-entry decode). Metric: decode layer-steps/s (one
+layer-step = one layer's decode step for the whole batch) and achieved HBM GB/s over the
+algorithmic bytes (indexer keys read + gathered MXFP4 codes and scales + FP8 SWA rows).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+With --gpus N > 1 run under torchrun: every rank decodes its own batch (data parallel, no
+collective on the data path); the step time is the max over ranks.
+--impl reference times the CPU oracle (a plain restatement of the same definitions) on a bounded
+sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import dataclasses
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "decode layer-steps/s and achieved HBM GB/s (% of 8 TB/s) at 1M ctx, 1 B200"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOADS = {w.name: w for w in (workloads.TINY, workloads.STACK3, workloads.PATTERN8,
+                                  workloads.MILLION)}
+DEFAULT = workloads.MILLION.name
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(wl) -> dict:
+    """Bytes the step must move (indexer keys + gathered MXFP4 entries + scales + SWA rows)."""
+    full = wl.B * wl.N * 128
+    reindex = wl.B * min(wl.P * 8, wl.N) * 128
+    attend = wl.B * (min(wl.K, wl.N) * 288 + wl.W * 516)
+    n_f = sum(m == "F" for m in wl.modes)
+    n_ri = sum(m == "RI" for m in wl.modes)
+    return dict(full=full, reindex=reindex, attend=attend,
+                step=n_f * full + n_ri * reindex + wl.L * attend)
+
+
+# --------------------------------------------------------------------------------- distributed
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value: float, dev) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(p[1]), smax=float(p[2]), power=float(p[3]),
+                                 active=p[4], hw=p[5], hwt=p[6], swt=p[7], pcap=p[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [r for r in rows if r["power"] > 200] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["smax"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# --------------------------------------------------------------------------------- our arm
+
+class Stack:
+    """Device state and the step of one CSA2 layer stack decoding a batch."""
+
+    def __init__(self, wl, dev):
+        import sparse_attention_decode_kv_b200 as csa2
+        self.csa2, self.wl, self.dev = csa2, wl, dev
+        B, K, P, W = wl.B, wl.K, wl.P, wl.W
+        self.n_cap = wl.n_cap
+        self.cache = csa2.Cache(B, self.n_cap, W, device=dev)
+        self._fill()
+        self.N = torch.full((B,), wl.N, dtype=torch.int32, device=dev)
+        self.swa_len = torch.full((B,), min(wl.N, W), dtype=torch.int32, device=dev)
+        self.pos_new = torch.full((B,), wl.N - 1, dtype=torch.int32, device=dev)
+        si = workloads.step_inputs(wl, dev)
+        self.q, self.iq, self.w = si["q"].contiguous(), si["iq"].contiguous(), si["w"].contiguous()
+        x_new, ik_new = workloads.new_token(wl, dev)
+        self.x_new, self.ik_new = x_new.contiguous(), ik_new.contiguous()
+        self.topk = torch.empty(wl.n_idx, B, K, dtype=torch.int32, device=dev)
+        self.pool = torch.empty(B, P * 8, dtype=torch.int32, device=dev)
+        self.out = torch.empty(wl.L, B, 16, 512, dtype=torch.float32, device=dev)
+        self.lse = torch.empty(wl.L, B, 16, dtype=torch.float32, device=dev)
+        self.ws_full = csa2.workspace(csa2.index_full_workspace_bytes(B, self.n_cap, K, P), dev)
+        self.ws_re = csa2.workspace(csa2.index_reindex_workspace_bytes(B, P * 8, K), dev)
+        self.ws_att = csa2.workspace(csa2.attend_workspace_bytes(B, K, W), dev)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def _fill(self):
+        wl, dev, csa2 = self.wl, self.dev, self.csa2
+        si = workloads.step_inputs(wl, dev)
+        pdirs = [workloads.plant_direction(si["iq"][0, b], si["w"][0, b]) if wl.n_planted else None
+                 for b in range(wl.B)]
+        for c in range(workloads.n_chunks(wl)):
+            x = torch.stack([workloads.kv_chunk(wl, b, c, dev) for b in range(wl.B)])
+            ik = torch.stack([workloads.ik_chunk(wl, b, c, dev, pdirs[b]) for b in range(wl.B)])
+            pos = torch.full((wl.B,), c * workloads.CHUNK, dtype=torch.int32, device=dev)
+            self.cache.append(x, ik, pos)
+            del x, ik
+        torch.cuda.synchronize()
+
+    # pieces of the step
+    def append_new(self):
+        self.cache.append(self.x_new, self.ik_new, self.pos_new, self.dev_err)
+
+    def index_full(self):
+        c = self.csa2
+        c.index_full(self.iq[0], self.w[0], self.cache.ik, self.N, self.wl.K, self.wl.P,
+                     self.topk[0], self.pool, self.ws_full, self.dev_err)
+
+    def layers(self):
+        """Everything after the Full index: Reindex layers and every layer's attention."""
+        c, wl, cache = self.csa2, self.wl, self.cache
+        j = 0
+        cur = None
+        for l, m in enumerate(wl.modes):
+            if m == "F":
+                cur = self.topk[j]
+                j += 1
+                mode = c.MODE_FULL
+            elif m == "RI":
+                c.index_reindex(self.iq[j], self.w[j], cache.ik, self.N, self.pool, wl.K,
+                                self.topk[j], self.ws_re, self.dev_err)
+                cur = self.topk[j]
+                j += 1
+                mode = c.MODE_REINDEX
+            else:
+                mode = c.MODE_REUSE
+            c.attend(mode, self.q[l], wl.softmax_scale, cache.codes, cache.scales, self.N, cur,
+                     cache.swa, cache.swa_scale, self.swa_len, self.out[l], self.lse[l],
+                     self.ws_att, self.dev_err)
+
+    def eager_step(self):
+        self.append_new()
+        self.index_full()
+        self.layers()
+
+
+def run_ours(args, world, rank, local):
+    import sparse_attention_decode_kv_b200 as csa2
+    from sparse_attention_decode_kv_b200 import build as csa2_build
+    if rank == 0:
+        csa2_build.build()
+    barrier(world)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    base = WORKLOADS[args.workload]
+    wl = dataclasses.replace(base, seed=base.seed + 1000 * rank)
+    st = Stack(wl, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # warm-up (eager), then capture the parts around the Full index into CUDA graphs; the Full
+    # index call is launched eagerly each step so that its scan kernel gets its own events
+    launches0 = csa2.launch_count()
+    st.eager_step()
+    torch.cuda.synchronize()
+    per_step_launches = csa2.launch_count() - launches0
+    g_app, g_layers = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_app, stream=torch.cuda.Stream(dev)):
+        st.append_new()
+    with torch.cuda.graph(g_layers, stream=torch.cuda.Stream(dev)):
+        st.layers()
+    torch.cuda.synchronize()
+
+    K, W = args.steps, args.warmup
+    ev_scan = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+    L = csa2.lib()
+
+    def step(i=None):
+        g_app.replay()
+        if i is not None:
+            L.csa2_set_profile_events(1, ctypes.c_void_p(ev_scan[i][0].cuda_event),
+                                      ctypes.c_void_p(ev_scan[i][1].cuda_event))
+        st.index_full()
+        if i is not None:
+            L.csa2_set_profile_events(1, None, None)
+        g_layers.replay()
+
+    for e in ev_scan:  # materialise the event handles
+        e[0].record(stream)
+        e[1].record(stream)
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(K):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms_local = t0.elapsed_time(t1)
+    ms = max_over_ranks(world, ms_local, dev)
+    scan_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_scan)
+    err = int(st.dev_err.item())
+    if err:
+        raise RuntimeError(f"device error flags {err:#x} during the benchmark")
+
+    ab = algorithmic_bytes(wl)
+    ms_step = ms / K
+    value = world * wl.L * K / (ms / 1e3)
+    achieved_step_gbs = world * ab["step"] * K / (ms / 1e3) / 1e9
+    peak, peak_kind = measured_peak()
+    scan_gbs = ab["full"] / (scan_ms / 1e3) / 1e9
+
+    e2e = None if args.no_e2e else run_e2e(st, step, K, W, world, dev)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, dev, samples=wl.B)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "layer-steps/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16/fp16-in fp32-acc (mxfp4+fp8 cache)",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "B_per_gpu": wl.B, "N": wl.N, "layers": ",".join(wl.modes),
+                   "K": wl.K, "P": wl.P, "W": wl.W, "cuda_graph": "append+layers; Full index eager",
+                   "l2": "inputs larger than L2 (indexer keys %.2f GB per step)" % (ab["full"] / 1e9),
+                   "parallelism": f"dp{world} (independent sequences)"},
+        "achieved_gbs": round(achieved_step_gbs, 1),
+        "pct_of_8TBs": round(100 * achieved_step_gbs / NOMINAL_HBM_GBS / world, 2),
+        "pct_of_measured_hbm": round(100 * achieved_step_gbs / peak / world, 2),
+        "sequence_layer_steps_per_s": round(value * wl.B, 1),
+        "roofline": {"kernel": "index_scan_kernel (Full-mode score scan)", "bound": "hbm",
+                     "achieved": round(scan_gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(scan_gbs / peak, 4), "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": ab["full"],
+                     "launch_ms": round(scan_ms, 4), "traffic": None},
+        "gpu_launches": per_step_launches * K,
+        "clocks": clocks.summary(),
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(st, step, K, W, world, dev):
+    """Same metric through the public API with host buffers: each step copies its inputs from
+    pinned host memory and reads its outputs back."""
+    stream = torch.cuda.current_stream(dev)
+    host_in = {name: t.detach().cpu().pin_memory() for name, t in
+               (("q", st.q), ("iq", st.iq), ("w", st.w), ("x_new", st.x_new),
+                ("ik_new", st.ik_new))}
+    host_out = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    host_lse = torch.empty(st.lse.shape, dtype=st.lse.dtype).pin_memory()
+    dev_in = {"q": st.q, "iq": st.iq, "w": st.w, "x_new": st.x_new, "ik_new": st.ik_new}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * 4 + host_lse.numel() * 4
+
+    def e2e_step():
+        for k, t in host_in.items():
+            dev_in[k].copy_(t, non_blocking=True)
+        step()
+        host_out.copy_(st.out, non_blocking=True)
+        host_lse.copy_(st.lse, non_blocking=True)
+
+    for _ in range(W):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(world, t0.elapsed_time(t1), dev)
+    return {"value": round(world * st.wl.L * K / (ms / 1e3), 2), "unit": "layer-steps/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms / K, 4)}
+
+
+# --------------------------------------------------------------------------------- oracle arm
+
+def oracle_sample_inputs(wl, dev, seqs):
+    """Host inputs for the oracle on sequences `seqs` of the workload (the same generators as the
+    GPU arm; nothing the CUDA kernels produced)."""
+    import numpy as np
+    si = workloads.step_inputs(wl, dev)
+    out = []
+    for b in seqs:
+        pdir = workloads.plant_direction(si["iq"][0, b], si["w"][0, b]) if wl.n_planted else None
+        ik = torch.cat([workloads.ik_chunk(wl, b, c, dev, pdir) for c in range(workloads.n_chunks(wl))])
+        out.append(dict(b=b, ik=workloads.bf16_bits(ik), q=workloads.bf16_bits(si["q"][:, b]),
+                        iq=workloads.bf16_bits(si["iq"][:, b]), w=si["w"][:, b].cpu().numpy()))
+    return out, np
+
+
+def oracle_rows(wl, b, rows, dev):
+    """bf16 main-KV rows `rows` of sequence b, regenerated chunk by chunk."""
+    import numpy as np
+    rows = np.asarray(rows, np.int64)
+    res = np.zeros((len(rows), 512), np.uint16)
+    for c in np.unique(rows // workloads.CHUNK):
+        m = rows // workloads.CHUNK == c
+        x = workloads.kv_chunk(wl, b, int(c), dev)
+        res[m] = workloads.bf16_bits(x[torch.as_tensor(rows[m] - c * workloads.CHUNK, device=dev)])
+    return res
+
+
+def oracle_one_sequence(wl, sample, dev):
+    """Time the oracle on one sequence's full stack step. Returns seconds of oracle compute (data
+    preparation between the index and attention parts is not timed)."""
+    import numpy as np
+
+    import oracle
+    N, K, P, W = wl.N, wl.K, wl.P, wl.W
+    ik = sample["ik"][None]
+    t_index = 0.0
+    topks = []
+    t = time.perf_counter()
+    r = oracle.index_full(sample["iq"][0][None], sample["w"][0][None], ik, [N], K, P)
+    t_index += time.perf_counter() - t
+    pool = r["pool"]
+    topks.append(r["topk"][0])
+    j = 1
+    per_layer = []
+    for m in wl.modes:
+        if m == "F":
+            per_layer.append(topks[0])
+        elif m == "RI":
+            t = time.perf_counter()
+            rr = oracle.index_reindex(sample["iq"][j][None], sample["w"][j][None], ik, pool, K)
+            t_index += time.perf_counter() - t
+            topks.append(rr["topk"][0])
+            per_layer.append(rr["topk"][0])
+            j += 1
+        else:
+            per_layer.append(per_layer[-1])
+    # untimed: the oracle quantises the rows the attention needs (remapped to a compact cache)
+    need = sorted(set(int(v) for tk in per_layer for v in tk if v >= 0))
+    rows = oracle_rows(wl, sample["b"], need, dev)
+    codes, scales = oracle.mxfp4_quantize(rows)
+    remap = {p: i for i, p in enumerate(need)}
+    swa_rows = oracle_rows(wl, sample["b"], list(range(N - min(N, W), N)), dev)
+    swa, swsc = oracle.swa_quantize(swa_rows)
+    # ring slot of position p is p mod W
+    ring = np.zeros((W, 512), np.uint8)
+    rsc = np.zeros((W,), np.float32)
+    for i, p in enumerate(range(N - min(N, W), N)):
+        ring[p % W], rsc[p % W] = swa[i], swsc[i]
+    t_att = 0.0
+    for l, tk in enumerate(per_layer):
+        idx = np.array([remap[int(v)] if v >= 0 else -1 for v in tk], np.int64)
+        t = time.perf_counter()
+        oracle.attend_seq(sample["q"][l], wl.softmax_scale, codes, scales, idx, ring, rsc, min(N, W))
+        t_att += time.perf_counter() - t
+    return t_index + t_att
+
+
+def cpu_baseline(wl, dev, samples=1):
+    seqs = list(range(min(samples, wl.B)))
+    inputs, _ = oracle_sample_inputs(wl, dev, seqs)
+    secs = [oracle_one_sequence(wl, s, dev) for s in inputs]
+    per_seq = statistics.mean(secs)
+    value = wl.L / (per_seq * wl.B)
+    return {"value": round(value, 4), "unit": "layer-steps/s", "cores": 1, "kind": "oracle",
+            "sample": (f"{len(seqs)} of {wl.B} sequences through all {wl.L} layers "
+                       f"(Full index over N={wl.N}, {sum(m == 'RI' for m in wl.modes)} Reindex, "
+                       f"{wl.L} attentions), scaled to the batch: {per_seq:.2f} s per sequence"),
+            "seconds": round(sum(secs), 2)}
+
+
+def run_reference(args, world, rank, local):
+    if rank != 0:
+        return
+    from oracle import build as oracle_build
+    oracle_build.build()
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    wl = WORKLOADS[args.workload]
+    inputs, _ = oracle_sample_inputs(wl, dev, [0])
+    for _ in range(args.warmup):
+        oracle_one_sequence(wl, inputs[0], dev)
+    secs = [oracle_one_sequence(wl, inputs[0], dev) for _ in range(args.steps)]
+    per_seq = statistics.mean(secs)
+    value = wl.L / (per_seq * wl.B)
+    sample = (f"sequence 0 of {wl.B} through all {wl.L} layers per step, scaled to the batch "
+              f"({per_seq:.2f} s per sequence)")
+    line = {"metric": METRIC, "value": round(value, 4), "unit": "layer-steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(per_seq * wl.B * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": wl.name, "B_per_gpu": wl.B, "N": wl.N,
+                       "layers": ",".join(wl.modes), "K": wl.K, "P": wl.P, "W": wl.W},
+            "cpu_baseline": {"value": round(value, 4), "unit": "layer-steps/s", "cores": 1,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "layer-steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank, local)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,448 @@
+// attend.cu -- sparse attention of one decode query per sequence (16 heads x 512) over the
+// selected MXFP4 main-KV entries and the FP8 SWA rows, merged into one softmax.
+//
+// Method: "DeepSeek V4.1 Flash 拆解" (austincafe.tech), section 一: a Reuse-mode layer reuses the
+// indices and runs sparse attention directly; the main KV is MXFP4, the SWA KV stays FP8.
+// Reading: K = V = the dequantised entry; z = softmax_scale * q . v over the selected entries and
+// the valid SWA slots together; out = sum softmax(z) v; lse = log sum exp(z).
+//
+// Work split: the K index slots and the W SWA slots are cut into tiles of 64 items (index tiles
+// and SWA tiles never mix); grid = (splits, B) and each CTA runs an online softmax over a
+// contiguous run of tiles. With one split the CTA writes the result; otherwise it writes an
+// unnormalised partial (m, l, o) and attend_merge_kernel combines the partials by log-sum-exp.
+//
+// Per tile: 16 threads per item gather 16-byte pieces (coalesced 256 B of codes + 32 B of scales
+// per MXFP4 entry, 512 B per SWA row), dequantise in registers with the sm_100a e2m1x2/e4m3x2 ->
+// f16x2 converts, and store an fp16 tile [64 x 512] in swizzled shared memory. Every dequantised
+// MXFP4 value (<= 6 significant bits, magnitude in [2^-10, 2688]) and every E4M3 element is exact
+// in fp16. QK^T and PV run on the tensor cores (m16n8k16, heads on M = 16, fp32 accumulate).
+// q is scaled per head by a power of two into fp16's range (exact for bf16 inputs). The SWA
+// per-token fp32 scale multiplies the logit and the probability instead of the value, so the
+// value operand stays exact; P is rescaled per SWA tile by a power of two to stay in fp16's
+// normal range.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace csa2 {
+
+namespace {
+
+constexpr int kTile = 64;
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kTargetCtas = 296;  // 148 SMs x 2 resident CTAs
+
+struct __align__(16) AttendSmem {
+  uint16_t q[HQ * D];        // fp16 [16][512], 16-byte chunks XOR-swizzled by (row & 7)
+  uint16_t v[kTile * D];     // fp16 [64][512], same swizzle
+  uint16_t p[HQ * kTile];    // fp16 [16][64], same swizzle (8 chunks per row)
+  float z[HQ * kTile];       // logits of the current tile
+  float item_scale[kTile];   // 1 (MXFP4) or the SWA token's fp32 scale
+  int item_valid[kTile];
+  float q_unscale[HQ];       // 2^(e_h - 14) * softmax_scale
+  float m_run[HQ], l_run[HQ], alpha[HQ];
+  float tile_pf;             // power of two applied to P on SWA tiles
+};
+
+__device__ __forceinline__ uint32_t swz1024(int row, int chunk) {  // 64 chunks per row
+  return static_cast<uint32_t>(row * 1024 + ((chunk ^ (row & 7)) << 4));
+}
+__device__ __forceinline__ uint32_t swz128(int row, int chunk) {  // 8 chunks per row
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+// 2^k as a float for k in [-126, 127].
+__device__ __forceinline__ float pow2f(int k) {
+  k = max(-126, min(127, k));
+  return __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
+}
+
+// floor(log2(x)) for finite x > 0 (subnormals clamp to -126).
+__device__ __forceinline__ int ilog2f(float x) {
+  const int e = static_cast<int>((__float_as_uint(x) >> 23) & 0xFF);
+  return e == 0 ? -126 : e - 127;
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+    attend_kernel(const uint16_t* __restrict__ q, float softmax_scale,
+                  const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                  int n_cap, const int32_t* __restrict__ N, const int32_t* __restrict__ idx, int K,
+                  const uint8_t* __restrict__ swa, const float* __restrict__ swa_scale,
+                  const int32_t* __restrict__ swa_len, int W, float* __restrict__ out,
+                  float* __restrict__ lse, float* __restrict__ part_o,
+                  float* __restrict__ part_ml, int32_t* dev_err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  AttendSmem& sm = *reinterpret_cast<AttendSmem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, c = lane & 3;
+  const int b = blockIdx.y, split = blockIdx.x, nsplit = gridDim.x;
+
+  const int tiles_idx = (K + kTile - 1) / kTile;
+  const int tiles_swa = (W + kTile - 1) / kTile;
+  const int tiles = tiles_idx + tiles_swa;
+  const int t_begin = static_cast<int>(static_cast<int64_t>(split) * tiles / nsplit);
+  const int t_end = static_cast<int>(static_cast<int64_t>(split + 1) * tiles / nsplit);
+
+  int nb = __ldg(N + b);
+  if (nb < 0 || nb > n_cap) {
+    if (tid == 0) flag_error(dev_err, CSA2_DEVERR_NLEN);
+    nb = max(0, min(nb, n_cap));
+  }
+  int sl = 0;
+  if (W > 0) {
+    sl = swa_len ? __ldg(swa_len + b) : 0;
+    if (sl < 0 || sl > W) {
+      if (tid == 0) flag_error(dev_err, CSA2_DEVERR_NLEN);
+      sl = max(0, min(sl, W));
+    }
+  }
+
+  // ---- q -> fp16 with a per-head power-of-two scale (16 threads per head, 32 dims each)
+  {
+    const int h = tid >> 4, r = tid & 15;
+    const uint4* src = reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * HQ + h) * D) +
+                       4 * r;
+    uint4 u[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u[k] = __ldg(src + k);
+    float amax = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t w4[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w4[e])), fabsf(bf16hi(w4[e]))));
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+    const int eh = amax > 0.0f ? ilog2f(amax) : 0;
+    const float up = pow2f(14 - eh);
+    if (r == 0) {
+      sm.q_unscale[h] = pow2f(eh - 14) * softmax_scale;
+      sm.m_run[h] = -INFINITY;
+      sm.l_run[h] = 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t w4[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+      uint32_t h2[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        __half2 hv = __floats2half2_rn(bf16lo(w4[e]) * up, bf16hi(w4[e]) * up);
+        h2[e] = *reinterpret_cast<uint32_t*>(&hv);
+      }
+      *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(sm.q) + swz1024(h, 4 * r + k)) =
+          make_uint4(h2[0], h2[1], h2[2], h2[3]);
+    }
+  }
+
+  float o[8][4];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
+
+  const uint32_t q_base = smem_u32(sm.q), v_base = smem_u32(sm.v), p_base = smem_u32(sm.p);
+  const int64_t seq_row0 = static_cast<int64_t>(b) * n_cap;
+
+  for (int tile = t_begin; tile < t_end; ++tile) {
+    const bool is_swa = tile >= tiles_idx;
+    const int base = is_swa ? (tile - tiles_idx) * kTile : tile * kTile;
+    const int count = min(kTile, (is_swa ? W : K) - base);
+
+    // ---- gather + dequantise: 16 threads per item, 32 channels per thread, 4 passes of 16 items
+    {
+      const int r = tid & 15;
+#pragma unroll
+      for (int pass = 0; pass < 4; ++pass) {
+        const int item = pass * 16 + (tid >> 4);
+        bool valid = false;
+        uint32_t hv[16];
+        float iscale = 1.0f;
+        if (item < count) {
+          if (!is_swa) {
+            const int pos = __ldg(idx + static_cast<int64_t>(b) * K + base + item);
+            if (pos >= 0 && pos < nb) {
+              valid = true;
+              const int64_t row = seq_row0 + pos;
+              const uint4 cw = ldg_nc_v4(codes + row * (D / 2) + 16 * r);
+              const uint32_t sw = __ldg(reinterpret_cast<const uint16_t*>(scales + row * (D / 16)) + r);
+              const uint32_t s01 = e4m3x2_to_h2(sw);  // .x = scale of channels 32r..+15, .y = next
+              const uint32_t slo = __byte_perm(s01, 0, 0x1010), shi = __byte_perm(s01, 0, 0x3232);
+              const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+              for (int k = 0; k < 16; ++k) {
+                const uint32_t byte = (cws[k >> 2] >> (8 * (k & 3))) & 0xFFu;
+                hv[k] = h2_mul(e2m1x2_to_h2(byte), k < 8 ? slo : shi);
+              }
+            } else if (pos != -1) {
+              flag_error(dev_err, CSA2_DEVERR_INDEX_RANGE);
+            }
+          } else {
+            const int slot = base + item;
+            if (slot < sl) {
+              valid = true;
+              const uint8_t* rowp = swa + (static_cast<int64_t>(b) * W + slot) * D + 32 * r;
+              const uint4 e0 = ldg_nc_v4(rowp), e1 = ldg_nc_v4(rowp + 16);
+              const uint32_t ew[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                hv[2 * k] = e4m3x2_to_h2(ew[k] & 0xFFFFu);
+                hv[2 * k + 1] = e4m3x2_to_h2(ew[k] >> 16);
+              }
+              iscale = __ldg(swa_scale + static_cast<int64_t>(b) * W + slot);
+            }
+          }
+        }
+        if (!valid) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) hv[k] = 0u;
+        }
+        unsigned char* vrow = reinterpret_cast<unsigned char*>(sm.v);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint4*>(vrow + swz1024(item, 4 * r + k)) =
+              make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
+        if (r == 0) {
+          sm.item_valid[item] = valid;
+          sm.item_scale[item] = iscale;
+        }
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // P scale for SWA tiles: brings the largest token scale to [1, 2)
+      float smax = 0.0f;
+      if (is_swa) {
+        smax = fmaxf(sm.item_valid[lane] ? sm.item_scale[lane] : 0.0f,
+                     sm.item_valid[lane + 32] ? sm.item_scale[lane + 32] : 0.0f);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xFFFFFFFFu, smax, off));
+      }
+      if (lane == 0) sm.tile_pf = smax > 0.0f ? pow2f(-ilog2f(smax)) : 1.0f;
+    }
+
+    // ---- logits: warp w computes z[0..16)[8w .. 8w+8)
+    {
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      const int mi = lane >> 3;
+      const int a_row = (lane & 7) + ((mi & 1) << 3);
+      const int v_row = 8 * warp + (lane & 7);
+#pragma unroll 4
+      for (int s = 0; s < D / 16; s += 2) {
+        uint32_t a0, a1, a2, a3, a4, a5, a6, a7, b0, b1, b2, b3;
+        ldsm_x4(q_base + swz1024(a_row, 2 * s + (mi >> 1)), a0, a1, a2, a3);
+        ldsm_x4(q_base + swz1024(a_row, 2 * s + 2 + (mi >> 1)), a4, a5, a6, a7);
+        ldsm_x4(v_base + swz1024(v_row, 2 * s + mi), b0, b1, b2, b3);
+        mma_f16_16816(acc, a0, a1, a2, a3, b0, b1);
+        mma_f16_16816(acc, a4, a5, a6, a7, b2, b3);
+      }
+      const int i0 = 8 * warp + 2 * c, i1 = i0 + 1;
+      const float u0 = sm.q_unscale[g], u1 = sm.q_unscale[g + 8];
+      const float s0 = sm.item_scale[i0], s1 = sm.item_scale[i1];
+      const bool v0 = sm.item_valid[i0], v1 = sm.item_valid[i1];
+      sm.z[g * kTile + i0] = v0 ? acc[0] * u0 * s0 : -INFINITY;
+      sm.z[g * kTile + i1] = v1 ? acc[1] * u0 * s1 : -INFINITY;
+      sm.z[(g + 8) * kTile + i0] = v0 ? acc[2] * u1 * s0 : -INFINITY;
+      sm.z[(g + 8) * kTile + i1] = v1 ? acc[3] * u1 * s1 : -INFINITY;
+    }
+    __syncthreads();
+
+    // ---- online softmax: warp w updates heads 2w and 2w+1
+    {
+      const float pf = sm.tile_pf;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int h = 2 * warp + hh;
+        const float z0 = sm.z[h * kTile + lane], z1 = sm.z[h * kTile + lane + 32];
+        float mt = fmaxf(z0, z1);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, off));
+        const float m_old = sm.m_run[h];
+        const float m_new = fmaxf(m_old, mt);
+        float p0 = 0.0f, p1 = 0.0f, alpha = 1.0f;
+        if (m_new != -INFINITY) {
+          p0 = __expf(z0 - m_new);
+          p1 = __expf(z1 - m_new);
+          alpha = __expf(m_old - m_new);
+        }
+        float ps = p0 + p1;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, off);
+        const float w0 = p0 * sm.item_scale[lane] * pf, w1 = p1 * sm.item_scale[lane + 32] * pf;
+        unsigned char* prow = reinterpret_cast<unsigned char*>(sm.p);
+        *reinterpret_cast<__half*>(prow + swz128(h, lane >> 3) + 2 * (lane & 7)) = __float2half_rn(w0);
+        *reinterpret_cast<__half*>(prow + swz128(h, 4 + (lane >> 3)) + 2 * (lane & 7)) =
+            __float2half_rn(w1);
+        if (lane == 0) {
+          sm.l_run[h] = sm.l_run[h] * alpha + ps;
+          sm.m_run[h] = m_new;
+          sm.alpha[h] = alpha;
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- o[16 heads][64w .. 64w+64) = alpha * o + P V  (pf undone after the MMAs)
+    {
+      const float pf = sm.tile_pf;
+      const float f0 = sm.alpha[g] * pf, f1 = sm.alpha[g + 8] * pf;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        o[j][0] *= f0;
+        o[j][1] *= f0;
+        o[j][2] *= f1;
+        o[j][3] *= f1;
+      }
+      const int mi = lane >> 3;
+      const int a_row = (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+      for (int s = 0; s < kTile / 16; ++s) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(p_base + swz128(a_row, 2 * s + (mi >> 1)), a0, a1, a2, a3);
+        const int v_row = 16 * s + (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_trans(v_base + swz1024(v_row, 8 * warp + j + (mi >> 1)), b0, b1, b2, b3);
+          mma_f16_16816(o[j], a0, a1, a2, a3, b0, b1);
+          mma_f16_16816(o[j + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+      if (pf != 1.0f) {
+        const float inv = 1.0f / pf;  // exact: pf is a power of two
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          o[j][0] *= inv;
+          o[j][1] *= inv;
+          o[j][2] *= inv;
+          o[j][3] *= inv;
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- epilogue: thread holds heads g and g+8, dims 64w + 8j + 2c (+1)
+  const float l0 = sm.l_run[g], l1 = sm.l_run[g + 8];
+  if (nsplit == 1) {
+    const float r0 = l0 > 0.0f ? 1.0f / l0 : 0.0f, r1 = l1 > 0.0f ? 1.0f / l1 : 0.0f;
+    float* o0 = out + (static_cast<int64_t>(b) * HQ + g) * D + 64 * warp + 2 * c;
+    float* o1 = out + (static_cast<int64_t>(b) * HQ + g + 8) * D + 64 * warp + 2 * c;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      *reinterpret_cast<float2*>(o0 + 8 * j) = make_float2(o[j][0] * r0, o[j][1] * r0);
+      *reinterpret_cast<float2*>(o1 + 8 * j) = make_float2(o[j][2] * r1, o[j][3] * r1);
+    }
+    if (lse != nullptr && tid < HQ) {
+      const float l = sm.l_run[tid];
+      lse[static_cast<int64_t>(b) * HQ + tid] = l > 0.0f ? sm.m_run[tid] + logf(l) : -INFINITY;
+    }
+  } else {
+    const int64_t pidx = static_cast<int64_t>(b) * nsplit + split;
+    float* o0 = part_o + (pidx * HQ + g) * D + 64 * warp + 2 * c;
+    float* o1 = part_o + (pidx * HQ + g + 8) * D + 64 * warp + 2 * c;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      *reinterpret_cast<float2*>(o0 + 8 * j) = make_float2(o[j][0], o[j][1]);
+      *reinterpret_cast<float2*>(o1 + 8 * j) = make_float2(o[j][2], o[j][3]);
+    }
+    if (tid < HQ) {
+      part_ml[(pidx * HQ + tid) * 2] = sm.m_run[tid];
+      part_ml[(pidx * HQ + tid) * 2 + 1] = sm.l_run[tid];
+    }
+  }
+}
+
+// Log-sum-exp merge of the split partials: grid = B, 16 threads per head, 32 dims per thread.
+__global__ void __launch_bounds__(256)
+    attend_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
+                        int nsplit, float* __restrict__ out, float* __restrict__ lse) {
+  const int b = blockIdx.x, h = threadIdx.x >> 4, r = threadIdx.x & 15;
+  const int64_t p0 = static_cast<int64_t>(b) * nsplit;
+  float m = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) m = fmaxf(m, part_ml[((p0 + s) * HQ + h) * 2]);
+  float l = 0.0f;
+  float acc[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) acc[k] = 0.0f;
+  if (m != -INFINITY) {
+    for (int s = 0; s < nsplit; ++s) {
+      const float ms = part_ml[((p0 + s) * HQ + h) * 2], ls = part_ml[((p0 + s) * HQ + h) * 2 + 1];
+      if (ms == -INFINITY) continue;
+      const float f = __expf(ms - m);
+      l += f * ls;
+      const float4* src = reinterpret_cast<const float4*>(part_o + ((p0 + s) * HQ + h) * D + 32 * r);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float4 v = src[k];
+        acc[4 * k] += f * v.x;
+        acc[4 * k + 1] += f * v.y;
+        acc[4 * k + 2] += f * v.z;
+        acc[4 * k + 3] += f * v.w;
+      }
+    }
+  }
+  const float rl = l > 0.0f ? 1.0f / l : 0.0f;
+  float4* dst = reinterpret_cast<float4*>(out + (static_cast<int64_t>(b) * HQ + h) * D + 32 * r);
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    dst[k] = make_float4(acc[4 * k] * rl, acc[4 * k + 1] * rl, acc[4 * k + 2] * rl,
+                         acc[4 * k + 3] * rl);
+  if (lse != nullptr && r == 0) lse[static_cast<int64_t>(b) * HQ + h] = l > 0.0f ? m + logf(l) : -INFINITY;
+}
+
+}  // namespace
+
+int attend_split_count(int B, int K, int W) {
+  const int tiles = (K + kTile - 1) / kTile + (W + kTile - 1) / kTile;
+  int splits = (kTargetCtas + B - 1) / B;
+  if (splits > tiles) splits = tiles;
+  if (splits < 1) splits = 1;
+  return splits;
+}
+
+size_t attend_workspace_bytes(int B, int K, int W) {
+  const int splits = attend_split_count(B, K, W);
+  if (splits == 1) return 0;
+  return static_cast<size_t>(B) * splits * HQ * (D + 2) * sizeof(float);
+}
+
+cudaError_t launch_attend(const void* q, float softmax_scale, const uint8_t* codes,
+                          const uint8_t* scales, int n_cap, const int32_t* N, const int32_t* idx,
+                          int K, const uint8_t* swa, const float* swa_scale,
+                          const int32_t* swa_len, int W, int B, float* out, float* lse, void* ws,
+                          int32_t* dev_err, cudaStream_t s) {
+  const int splits = attend_split_count(B, K, W);
+  float* part_o = nullptr;
+  float* part_ml = nullptr;
+  if (splits > 1) {
+    part_o = static_cast<float*>(ws);
+    part_ml = part_o + static_cast<size_t>(B) * splits * HQ * D;
+  }
+  const size_t smem = sizeof(AttendSmem);
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  profile_begin(CSA2_KERNEL_ATTEND, s);
+  attend_kernel<<<dim3(splits, B), kThreads, smem, s>>>(
+      static_cast<const uint16_t*>(q), softmax_scale, codes, scales, n_cap, N, idx, K, swa,
+      swa_scale, swa_len, W, out, lse, part_o, part_ml, dev_err);
+  count_launches(1);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess && splits > 1) {
+    attend_merge_kernel<<<B, 256, 0, s>>>(part_o, part_ml, splits, out, lse);
+    count_launches(1);
+    e = cudaGetLastError();
+  }
+  profile_end(CSA2_KERNEL_ATTEND, s);
+  return e;
+}
+
+}  // namespace csa2

@@ -1,0 +1,43 @@
+// internal.h -- host-side launchers behind the C ABI (not part of the public interface).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace csa2 {
+
+void count_launches(int n);   // adds to the process-wide launch counter
+void profile_begin(int kernel, cudaStream_t s);  // records the start event if one is set
+void profile_end(int kernel, cudaStream_t s);    // records the stop event if one is set
+int device_sm_count();        // SMs of the current device (cached per device)
+
+// Quantize-on-append; one warp per new entry.
+cudaError_t launch_append(const void* x, const void* ik, int B, int n, const int32_t* pos,
+                          int n_cap, uint8_t* codes, uint8_t* scales, void* ik_cache,
+                          uint8_t* swa, float* swa_scale, int W, int32_t* dev_err,
+                          cudaStream_t s);
+
+// Sparse attention (split over item tiles, merged by log-sum-exp).
+size_t attend_workspace_bytes(int B, int K, int W);
+int attend_split_count(int B, int K, int W);
+cudaError_t launch_attend(const void* q, float softmax_scale, const uint8_t* codes,
+                          const uint8_t* scales, int n_cap, const int32_t* N, const int32_t* idx,
+                          int K, const uint8_t* swa, const float* swa_scale,
+                          const int32_t* swa_len, int W, int B, float* out, float* lse, void* ws,
+                          int32_t* dev_err, cudaStream_t s);
+
+// Full-mode indexer.
+size_t index_full_workspace_bytes(int B, int n_cap, int K, int P);
+cudaError_t launch_index_full(const void* iq, const float* w, const void* ik_cache,
+                              const int32_t* N, int B, int n_cap, int K, int P, int32_t* topk,
+                              int32_t* pool, void* ws, int32_t* dev_err, cudaStream_t s);
+
+// Reindex-mode indexer.
+size_t index_reindex_workspace_bytes(int B, int L, int K);
+cudaError_t launch_index_reindex(const void* iq, const float* w, const void* ik_cache,
+                                 const int32_t* N, int B, int n_cap, const int32_t* pool, int L,
+                                 int K, int32_t* topk, void* ws, int32_t* dev_err,
+                                 cudaStream_t s);
+
+}  // namespace csa2
