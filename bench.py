@@ -47,12 +47,14 @@ DEFAULT = workloads.MILLION.name
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--breakdown", action="store_true",
+                    help="also time each library call of the step (eager, synchronised)")
     return ap.parse_args()
 
 
@@ -97,12 +99,25 @@ def barrier(world):
 
 
 def max_over_ranks(world, value: float, dev) -> float:
+    """The slowest rank's time (an NCCL all-reduce on the device; gloo uses the host)."""
     if world == 1:
         return value
     import torch.distributed as dist
+    if dist.get_backend() == "gloo":
+        dev = torch.device("cpu")
     t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(base, rank: int):
+    """Data parallel: every rank decodes its own batch of independent sequences."""
+    return dataclasses.replace(base, seed=base.seed + 1000 * rank)
+
+
+def aggregate_value(world: int, layers: int, steps: int, ms_max: float) -> float:
+    """Whole-job layer-steps/s: every rank runs `layers` layer-steps per step."""
+    return world * layers * steps / (ms_max / 1e3)
 
 
 # --------------------------------------------------------------------------------- clocks
@@ -123,7 +138,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -254,7 +269,7 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     base = WORKLOADS[args.workload]
-    wl = dataclasses.replace(base, seed=base.seed + 1000 * rank)
+    wl = rank_workload(base, rank)
     st = Stack(wl, dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -313,12 +328,13 @@ def run_ours(args, world, rank, local):
 
     ab = algorithmic_bytes(wl)
     ms_step = ms / K
-    value = world * wl.L * K / (ms / 1e3)
+    value = aggregate_value(world, wl.L, K, ms)
     achieved_step_gbs = world * ab["step"] * K / (ms / 1e3) / 1e9
     peak, peak_kind = measured_peak()
     scan_gbs = ab["full"] / (scan_ms / 1e3) / 1e9
 
     e2e = None if args.no_e2e else run_e2e(st, step, K, W, world, dev)
+    parts = breakdown(st) if args.breakdown else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, dev, samples=wl.B)
@@ -346,10 +362,72 @@ def run_ours(args, world, rank, local):
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if parts is not None:
+        line["breakdown_us"] = parts
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def breakdown(st, steps=20):
+    """Median device time (us) of each library call of an eager step, from CUDA events recorded
+    around every call on the launching stream (diagnostic; not the headline number)."""
+    stream = torch.cuda.current_stream(st.dev)
+    L = st.csa2.lib()
+    parts = {}
+
+    def pair():
+        # torch creates the CUDA event on first record; record once so the handle exists
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        b.record(stream)
+        return a, b
+
+    def timed(name, kernel_id, fn):
+        a, b = pair()
+        L.csa2_set_profile_events(kernel_id, ctypes.c_void_p(a.cuda_event),
+                                  ctypes.c_void_p(b.cuda_event))
+        fn()
+        L.csa2_set_profile_events(kernel_id, None, None)
+        parts.setdefault(name, []).append((a, b))
+
+    wl, c, cache = st.wl, st.csa2, st.cache
+    samples = {}
+    for _ in range(steps):
+        parts.clear()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        timed("append", 0, st.append_new)
+        ev = [pair(), pair()]
+        L.csa2_set_profile_events(1, ctypes.c_void_p(ev[0][0].cuda_event), ctypes.c_void_p(ev[0][1].cuda_event))
+        L.csa2_set_profile_events(2, ctypes.c_void_p(ev[1][0].cuda_event), ctypes.c_void_p(ev[1][1].cuda_event))
+        st.index_full()
+        L.csa2_set_profile_events(1, None, None)
+        L.csa2_set_profile_events(2, None, None)
+        parts["index_scan"] = [ev[0]]
+        parts["index_select"] = [ev[1]]
+        j, cur = 0, None
+        for l, m in enumerate(wl.modes):
+            if m == "F":
+                cur, j, mode = st.topk[j], j + 1, c.MODE_FULL
+            elif m == "RI":
+                jj = j
+                timed("reindex", 3, lambda jj=jj: c.index_reindex(
+                    st.iq[jj], st.w[jj], cache.ik, st.N, st.pool, wl.K, st.topk[jj], st.ws_re,
+                    st.dev_err))
+                cur, j, mode = st.topk[j], j + 1, c.MODE_REINDEX
+            else:
+                mode = c.MODE_REUSE
+            timed("attend", 4, lambda l=l, mode=mode, cur=cur: c.attend(
+                mode, st.q[l], wl.softmax_scale, cache.codes, cache.scales, st.N, cur, cache.swa,
+                cache.swa_scale, st.swa_len, st.out[l], st.lse[l], st.ws_att, st.dev_err))
+        a1.record(stream)
+        torch.cuda.synchronize()
+        for name, evs in parts.items():
+            samples.setdefault(name, []).append(sum(x.elapsed_time(y) for x, y in evs) * 1e3)
+        samples.setdefault("eager_step", []).append(a0.elapsed_time(a1) * 1e3)
+    return {k: round(statistics.median(v), 2) for k, v in samples.items()}
 
 
 def run_e2e(st, step, K, W, world, dev):

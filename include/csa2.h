@@ -116,8 +116,9 @@ CSA2_API int csa2_append_quant(const void *x, const void *ik, int B, int n, cons
  *   topk      int32 [B, K] out: ascending positions, -1 padded when N[b] < K.
  *   pool      int32 [B, 8P] out: the selected blocks' positions (ascending block order), -1 for
  *             positions >= N[b] and for unused blocks.
- * The workspace starts with the fp32 scores I [B, n_cap] (valid for t < N[b]) followed by the
- * fp32 block maxima [B, n_cap/8]; both stay readable until the workspace is reused.
+ * Layout contract: the workspace starts with the fp32 scores I [B, n_cap] (valid for t < N[b]);
+ * the fp32 block maxima [B, n_cap/8] follow at byte offset 4*B*n_cap rounded up to a multiple of
+ * 256. Both stay readable until the workspace is reused.
  */
 CSA2_API size_t csa2_index_full_workspace_bytes(int B, int n_cap, int K, int P);
 CSA2_API int csa2_index_full(const void *iq, const float *w, const void *ik_cache, const int32_t *N, int B,

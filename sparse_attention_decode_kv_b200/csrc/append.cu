@@ -58,6 +58,8 @@ __global__ void __launch_bounds__(kAppendWarps * 32)
                   uint8_t* __restrict__ scales, uint16_t* __restrict__ ik_cache,
                   uint8_t* __restrict__ swa, float* __restrict__ swa_scale, int W,
                   int32_t* dev_err) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t entry = static_cast<int64_t>(blockIdx.x) * kAppendWarps + (threadIdx.x >> 5);
   if (entry >= static_cast<int64_t>(B) * n) return;
@@ -124,12 +126,13 @@ cudaError_t launch_append(const void* x, const void* ik, int B, int n, const int
   const int64_t blocks = (entries + kAppendWarps - 1) / kAppendWarps;
   if (blocks > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
   profile_begin(CSA2_KERNEL_APPEND, s);
-  append_kernel<<<static_cast<unsigned>(blocks), kAppendWarps * 32, 0, s>>>(
-      static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(ik), B, n, pos, n_cap, codes,
-      scales, static_cast<uint16_t*>(ik_cache), swa, swa_scale, W, dev_err);
+  cudaError_t e = launch_pdl(append_kernel, dim3(static_cast<unsigned>(blocks)),
+                             dim3(kAppendWarps * 32), 0, s, static_cast<const uint16_t*>(x),
+                             static_cast<const uint16_t*>(ik), B, n, pos, n_cap, codes, scales,
+                             static_cast<uint16_t*>(ik_cache), swa, swa_scale, W, dev_err);
   profile_end(CSA2_KERNEL_APPEND, s);
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace csa2

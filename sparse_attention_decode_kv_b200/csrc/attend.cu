@@ -78,6 +78,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, c = lane & 3;
   const int b = blockIdx.y, split = blockIdx.x, nsplit = gridDim.x;
+  pdl_wait();
+  pdl_launch_dependents();
 
   const int tiles_idx = (K + kTile - 1) / kTile;
   const int tiles_swa = (W + kTile - 1) / kTile;
@@ -150,62 +152,83 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int base = is_swa ? (tile - tiles_idx) * kTile : tile * kTile;
     const int count = min(kTile, (is_swa ? W : K) - base);
 
-    // ---- gather + dequantise: 16 threads per item, 32 channels per thread, 4 passes of 16 items
+    // ---- gather + dequantise: 16 threads per item, 32 channels per thread, 4 passes of 16 items.
+    // All index loads, then all row loads, then the conversions: two memory round trips.
     {
       const int r = tid & 15;
+      unsigned char* vrow = reinterpret_cast<unsigned char*>(sm.v);
+      if (!is_swa) {
+        int pos[4];
 #pragma unroll
-      for (int pass = 0; pass < 4; ++pass) {
-        const int item = pass * 16 + (tid >> 4);
-        bool valid = false;
-        uint32_t hv[16];
-        float iscale = 1.0f;
-        if (item < count) {
-          if (!is_swa) {
-            const int pos = __ldg(idx + static_cast<int64_t>(b) * K + base + item);
-            if (pos >= 0 && pos < nb) {
-              valid = true;
-              const int64_t row = seq_row0 + pos;
-              const uint4 cw = ldg_nc_v4(codes + row * (D / 2) + 16 * r);
-              const uint32_t sw = __ldg(reinterpret_cast<const uint16_t*>(scales + row * (D / 16)) + r);
-              const uint32_t s01 = e4m3x2_to_h2(sw);  // .x = scale of channels 32r..+15, .y = next
-              const uint32_t slo = __byte_perm(s01, 0, 0x1010), shi = __byte_perm(s01, 0, 0x3232);
-              const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+        for (int pass = 0; pass < 4; ++pass) {
+          const int item = pass * 16 + (tid >> 4);
+          pos[pass] = item < count ? __ldg(idx + static_cast<int64_t>(b) * K + base + item) : -1;
+        }
+        uint4 cw[4];
+        uint32_t sw[4];
 #pragma unroll
-              for (int k = 0; k < 16; ++k) {
-                const uint32_t byte = (cws[k >> 2] >> (8 * (k & 3))) & 0xFFu;
-                hv[k] = h2_mul(e2m1x2_to_h2(byte), k < 8 ? slo : shi);
-              }
-            } else if (pos != -1) {
-              flag_error(dev_err, CSA2_DEVERR_INDEX_RANGE);
-            }
-          } else {
-            const int slot = base + item;
-            if (slot < sl) {
-              valid = true;
-              const uint8_t* rowp = swa + (static_cast<int64_t>(b) * W + slot) * D + 32 * r;
-              const uint4 e0 = ldg_nc_v4(rowp), e1 = ldg_nc_v4(rowp + 16);
-              const uint32_t ew[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+        for (int pass = 0; pass < 4; ++pass) {
+          const bool valid = pos[pass] >= 0 && pos[pass] < nb;
+          if (!valid && pos[pass] != -1) flag_error(dev_err, CSA2_DEVERR_INDEX_RANGE);
+          const int64_t row = seq_row0 + (valid ? pos[pass] : 0);
+          cw[pass] = valid ? ldg_nc_v4(codes + row * (D / 2) + 16 * r) : make_uint4(0u, 0u, 0u, 0u);
+          sw[pass] = valid ? __ldg(reinterpret_cast<const uint16_t*>(scales + row * (D / 16)) + r) : 0u;
+        }
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                hv[2 * k] = e4m3x2_to_h2(ew[k] & 0xFFFFu);
-                hv[2 * k + 1] = e4m3x2_to_h2(ew[k] >> 16);
-              }
-              iscale = __ldg(swa_scale + static_cast<int64_t>(b) * W + slot);
-            }
+        for (int pass = 0; pass < 4; ++pass) {
+          const int item = pass * 16 + (tid >> 4);
+          const bool valid = pos[pass] >= 0 && pos[pass] < nb;
+          const uint32_t s01 = e4m3x2_to_h2(sw[pass]);  // .x: channels 32r..+15, .y: the next 16
+          const uint32_t slo = __byte_perm(s01, 0, 0x1010), shi = __byte_perm(s01, 0, 0x3232);
+          const uint32_t cws[4] = {cw[pass].x, cw[pass].y, cw[pass].z, cw[pass].w};
+          uint32_t hv[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const uint32_t byte = (cws[k >> 2] >> (8 * (k & 3))) & 0xFFu;
+            hv[k] = h2_mul(e2m1x2_to_h2(byte), k < 8 ? slo : shi);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4*>(vrow + swz1024(item, 4 * r + k)) =
+                make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
+          if (r == 0) {
+            sm.item_valid[item] = valid;
+            sm.item_scale[item] = 1.0f;
           }
         }
-        if (!valid) {
+      } else {
+        uint4 e[4][2];
+        float iscale[4];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) hv[k] = 0u;
+        for (int pass = 0; pass < 4; ++pass) {
+          const int item = pass * 16 + (tid >> 4);
+          const int slot = base + item;
+          const bool valid = item < count && slot < sl;
+          const uint8_t* rowp = swa + (static_cast<int64_t>(b) * W + (valid ? slot : 0)) * D + 32 * r;
+          e[pass][0] = valid ? ldg_nc_v4(rowp) : make_uint4(0u, 0u, 0u, 0u);
+          e[pass][1] = valid ? ldg_nc_v4(rowp + 16) : make_uint4(0u, 0u, 0u, 0u);
+          iscale[pass] = valid ? __ldg(swa_scale + static_cast<int64_t>(b) * W + slot) : 1.0f;
         }
-        unsigned char* vrow = reinterpret_cast<unsigned char*>(sm.v);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          *reinterpret_cast<uint4*>(vrow + swz1024(item, 4 * r + k)) =
-              make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
-        if (r == 0) {
-          sm.item_valid[item] = valid;
-          sm.item_scale[item] = iscale;
+        for (int pass = 0; pass < 4; ++pass) {
+          const int item = pass * 16 + (tid >> 4);
+          const bool valid = item < count && base + item < sl;
+          const uint32_t ew[8] = {e[pass][0].x, e[pass][0].y, e[pass][0].z, e[pass][0].w,
+                                  e[pass][1].x, e[pass][1].y, e[pass][1].z, e[pass][1].w};
+          uint32_t hv[16];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            hv[2 * k] = e4m3x2_to_h2(ew[k] & 0xFFFFu);
+            hv[2 * k + 1] = e4m3x2_to_h2(ew[k] >> 16);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4*>(vrow + swz1024(item, 4 * r + k)) =
+                make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
+          if (r == 0) {
+            sm.item_valid[item] = valid;
+            sm.item_scale[item] = iscale[pass];
+          }
         }
       }
     }
@@ -354,42 +377,65 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-// Log-sum-exp merge of the split partials: grid = B, 16 threads per head, 32 dims per thread.
-__global__ void __launch_bounds__(256)
+// Log-sum-exp merge of the split partials: grid = (16 heads, B), 128 threads x 4 dims. The
+// (m, l) pairs of all splits are read at once into shared memory, then every thread issues its
+// partial loads in groups of 8 independent requests.
+constexpr int kMaxSplits = 128;
+__global__ void __launch_bounds__(128)
     attend_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                         int nsplit, float* __restrict__ out, float* __restrict__ lse) {
-  const int b = blockIdx.x, h = threadIdx.x >> 4, r = threadIdx.x & 15;
+  __shared__ float wgt[kMaxSplits];
+  __shared__ float ml[2];
+  const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
   const int64_t p0 = static_cast<int64_t>(b) * nsplit;
-  float m = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) m = fmaxf(m, part_ml[((p0 + s) * HQ + h) * 2]);
-  float l = 0.0f;
-  float acc[32];
+  float ms = -INFINITY, ls = 0.0f;
+  if (t < nsplit) {
+    ms = __ldg(part_ml + ((p0 + t) * HQ + h) * 2);
+    ls = __ldg(part_ml + ((p0 + t) * HQ + h) * 2 + 1);
+  }
+  float m = ms;
 #pragma unroll
-  for (int k = 0; k < 32; ++k) acc[k] = 0.0f;
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+  if ((t & 31) == 0) wgt[t >> 5] = m;  // per-warp max (nsplit <= 128 = blockDim)
+  __syncthreads();
+  m = fmaxf(fmaxf(wgt[0], wgt[1]), fmaxf(wgt[2], wgt[3]));
+  __syncthreads();
+  const float f = (t < nsplit && ms != -INFINITY) ? __expf(ms - m) : 0.0f;
+  if (t < nsplit) wgt[t] = f;
+  float fl = f * ls;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) fl += __shfl_xor_sync(0xFFFFFFFFu, fl, off);
+  if (t == 0) ml[0] = 0.0f;
+  __syncthreads();
+  if ((t & 31) == 0) atomicAdd(&ml[0], fl);
+  __syncthreads();
+  const float l = ml[0];
+  float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   if (m != -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      const float ms = part_ml[((p0 + s) * HQ + h) * 2], ls = part_ml[((p0 + s) * HQ + h) * 2 + 1];
-      if (ms == -INFINITY) continue;
-      const float f = __expf(ms - m);
-      l += f * ls;
-      const float4* src = reinterpret_cast<const float4*>(part_o + ((p0 + s) * HQ + h) * D + 32 * r);
+    const float4* src = reinterpret_cast<const float4*>(part_o + (p0 * HQ + h) * D) + t;
+    const int64_t stride = static_cast<int64_t>(HQ) * D / 4;  // float4 between splits
+    for (int s0 = 0; s0 < nsplit; s0 += 8) {
+      float4 v[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float4 v = src[k];
-        acc[4 * k] += f * v.x;
-        acc[4 * k + 1] += f * v.y;
-        acc[4 * k + 2] += f * v.z;
-        acc[4 * k + 3] += f * v.w;
+      for (int j = 0; j < 8; ++j)
+        v[j] = s0 + j < nsplit ? __ldg(src + (s0 + j) * stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float fj = s0 + j < nsplit ? wgt[s0 + j] : 0.0f;
+        acc.x += fj * v[j].x;
+        acc.y += fj * v[j].y;
+        acc.z += fj * v[j].z;
+        acc.w += fj * v[j].w;
       }
     }
   }
   const float rl = l > 0.0f ? 1.0f / l : 0.0f;
-  float4* dst = reinterpret_cast<float4*>(out + (static_cast<int64_t>(b) * HQ + h) * D + 32 * r);
-#pragma unroll
-  for (int k = 0; k < 8; ++k)
-    dst[k] = make_float4(acc[4 * k] * rl, acc[4 * k + 1] * rl, acc[4 * k + 2] * rl,
-                         acc[4 * k + 3] * rl);
-  if (lse != nullptr && r == 0) lse[static_cast<int64_t>(b) * HQ + h] = l > 0.0f ? m + logf(l) : -INFINITY;
+  reinterpret_cast<float4*>(out + (static_cast<int64_t>(b) * HQ + h) * D)[t] =
+      make_float4(acc.x * rl, acc.y * rl, acc.z * rl, acc.w * rl);
+  if (lse != nullptr && t == 0)
+    lse[static_cast<int64_t>(b) * HQ + h] = l > 0.0f ? m + logf(l) : -INFINITY;
 }
 
 }  // namespace
@@ -398,6 +444,7 @@ int attend_split_count(int B, int K, int W) {
   const int tiles = (K + kTile - 1) / kTile + (W + kTile - 1) / kTile;
   int splits = (kTargetCtas + B - 1) / B;
   if (splits > tiles) splits = tiles;
+  if (splits > kMaxSplits) splits = kMaxSplits;
   if (splits < 1) splits = 1;
   return splits;
 }
@@ -431,15 +478,18 @@ cudaError_t launch_attend(const void* q, float softmax_scale, const uint8_t* cod
     configured_device = dev;
   }
   profile_begin(CSA2_KERNEL_ATTEND, s);
-  attend_kernel<<<dim3(splits, B), kThreads, smem, s>>>(
-      static_cast<const uint16_t*>(q), softmax_scale, codes, scales, n_cap, N, idx, K, swa,
-      swa_scale, swa_len, W, out, lse, part_o, part_ml, dev_err);
+  cudaError_t e = launch_pdl(attend_kernel, dim3(splits, B), dim3(kThreads), smem, s,
+                             static_cast<const uint16_t*>(q), softmax_scale, codes, scales, n_cap,
+                             N, idx, K, swa, swa_scale, swa_len, W, out, lse, part_o, part_ml,
+                             dev_err);
   count_launches(1);
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e == cudaSuccess && splits > 1) {
-    attend_merge_kernel<<<B, 256, 0, s>>>(part_o, part_ml, splits, out, lse);
+    e = launch_pdl(attend_merge_kernel, dim3(HQ, B), dim3(128), 0, s,
+                   static_cast<const float*>(part_o), static_cast<const float*>(part_ml), splits,
+                   out, lse);
     count_launches(1);
-    e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaGetLastError();
   }
   profile_end(CSA2_KERNEL_ATTEND, s);
   return e;

@@ -10,16 +10,21 @@
 // Full mode, three kernels on the caller's stream:
 //   index_scan_kernel   persistent, one CTA per SM. One producer thread streams 128-entry key
 //                       tiles (16 KiB, 128-byte swizzle) with cp.async.bulk.tensor into a
-//                       6-stage mbarrier ring; 8 consumer warps run the 4-head q.K contraction
-//                       on the tensor cores (m16n8k16 bf16, keys on M, heads padded to N = 8),
-//                       then ReLU, weights, fp32 score store, block max over 8 positions and
-//                       4096-bin histograms (top 12 key bits) of scores and block maxima.
-//   topk_collect_kernel every CTA finds the histogram bin holding the K-th score (P-th block)
-//                       and appends the rank keys of all items in or above that bin to a
-//                       candidate buffer (warp-aggregated atomics).
-//   topk_final_kernel   one CTA per (sequence, positions|blocks): exact radix select over the
-//                       candidates (or, if they overflowed, over the full score array), bitonic
-//                       sort of the winners by index, then topk / pool output.
+//                       6-stage mbarrier ring; two groups of 8 consumer warps take alternate
+//                       tiles and run the 4-head q.K contraction on the tensor cores (m16n8k16
+//                       bf16, keys on M, heads padded to N = 8), then ReLU, weights, the fp32
+//                       score store, the block max over 8 positions and a 4096-bin histogram
+//                       (top 12 key bits) of the block maxima.
+//   block_collect_kernel  finds the histogram bin holding the max(K, P)-th block and copies the
+//                       rank keys of all blocks in or above it, in block order, into one region
+//                       per 8192-block chunk.
+//   index_final_kernel  one CTA per sequence: radix select of the top max(K, P) blocks over the
+//                       candidates, order-preserving compaction (ascending block ids, no sort),
+//                       the pool (top P blocks), then the position Top-K over the scores of the
+//                       selected blocks' positions. Every Top-K position lies in one of the top
+//                       max(K, P) blocks: a block ranked above the block of a selected position
+//                       holds its own maximum, which outranks that position, so fewer than K
+//                       blocks outrank it.
 // Every mbarrier wait is bounded; a timeout flags CSA2_DEVERR_TIMEOUT and the CTA drains its own
 // bulk copies before exiting.
 #include <mutex>
@@ -36,23 +41,26 @@ namespace {
 constexpr int kScanTile = 128;                    // entries per TMA tile
 constexpr int kScanTileBytes = kScanTile * DI * 2;  // 16 KiB
 constexpr int kScanStages = 6;
-constexpr int kScanConsumerWarps = 8;             // 16 entries each per tile
+constexpr int kScanGroupWarps = 8;                // warps sharing one tile, 16 entries each
+constexpr int kScanConsumerWarps = 2 * kScanGroupWarps;  // two groups take alternate tiles
 constexpr int kScanThreads = (kScanConsumerWarps + 1) * 32;
-constexpr int kCand = 16384;                      // candidate slots per (sequence, problem)
-constexpr int kCollectChunk = 8192;
+constexpr int kCollectChunk = 8192;              // blocks per collect CTA (and per region)
 constexpr int kCollectThreads = 256;
 constexpr int kFinalThreads = 1024;
 constexpr int kMaxSel = 4096;                     // >= CSA2_MAX_K, CSA2_MAX_P
+constexpr int kSmemKeys = 16384;                  // candidate keys held in shared memory
 
 static_assert(kScanTileBytes == 16384, "tile size");
 
-struct __align__(1024) ScanSmem {
+struct __align__(1024) ScanSmem {  // checked against the 227 KiB limit below
   uint8_t tiles[kScanStages][kScanTileBytes];
   uint64_t full[kScanStages];
   uint64_t empty[kScanStages];
-  uint32_t hist[2][kHistBins];
+  uint32_t hist[kHistBins];  // block maxima
   int abort;
 };
+
+static_assert(sizeof(ScanSmem) <= 227 * 1024, "index_scan_kernel shared memory");
 
 __device__ __forceinline__ void consumer_bar() {
   asm volatile("bar.sync 1, %0;" ::"n"(kScanConsumerWarps * 32) : "memory");
@@ -89,12 +97,16 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   const int64_t total = static_cast<int64_t>(B) * tiles_per_seq;
   const int64_t v_begin = total * blockIdx.x / gridDim.x;
   const int64_t v_end = total * (blockIdx.x + 1) / gridDim.x;
+  const int n_tiles = static_cast<int>(v_end - v_begin);
+  // (sequence, tile) of the first virtual tile; later ones are walked incrementally
+  const int b_first = static_cast<int>(v_begin / tiles_per_seq);
+  const int t_first = static_cast<int>(v_begin - static_cast<int64_t>(b_first) * tiles_per_seq);
 
-  for (int i = tid; i < 2 * kHistBins; i += kScanThreads) (&sm.hist[0][0])[i] = 0u;
+  for (int i = tid; i < kHistBins; i += kScanThreads) sm.hist[i] = 0u;
   if (tid == 0) {
     for (int s = 0; s < kScanStages; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], kScanConsumerWarps);
+      mbar_init(&sm.empty[s], kScanGroupWarps);
     }
     sm.abort = 0;
     fence_barrier_init();
@@ -106,58 +118,68 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     // ------------------------------------------------------------------ producer (one thread)
     if (lane == 0) {
       const uint64_t policy = l2_policy_evict_first();
-      int64_t it = 0;
-      for (int64_t v = v_begin; v < v_end && !*abort; ++v) {
-        const int b = static_cast<int>(v / tiles_per_seq);
-        const int t = static_cast<int>(v - static_cast<int64_t>(b) * tiles_per_seq);
-        const int nb = max(0, min(__ldg(N + b), n_cap));
-        if (t * kScanTile >= nb) continue;
-        const int stage = static_cast<int>(it % kScanStages);
-        const int64_t round = it / kScanStages;
-        if (round > 0 && !wait_or_abort(&sm.empty[stage], static_cast<uint32_t>((round - 1) & 1), abort)) {
-          flag_error(dev_err, CSA2_DEVERR_TIMEOUT);
-          *abort = 1;
-          break;
+      int b = b_first, t = t_first, nb = max(0, min(__ldg(N + b), n_cap));
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      for (int k = 0; k < n_tiles && !*abort; ++k) {
+        if (t * kScanTile < nb) {
+          if (issued >= kScanStages && !wait_or_abort(&sm.empty[stage], phase ^ 1u, abort)) {
+            flag_error(dev_err, CSA2_DEVERR_TIMEOUT);
+            *abort = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.full[stage], kScanTileBytes);
+          tma_load_3d(sm.tiles[stage], &keys, &sm.full[stage], 0, t * kScanTile, b, policy);
+          ++issued;
+          if (++stage == kScanStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
-        mbar_arrive_expect_tx(&sm.full[stage], kScanTileBytes);
-        tma_load_3d(sm.tiles[stage], &keys, &sm.full[stage], 0, t * kScanTile, b, policy);
-        ++it;
+        if (++t == tiles_per_seq && k + 1 < n_tiles) {
+          t = 0;
+          ++b;
+          nb = max(0, min(__ldg(N + b), n_cap));
+        }
       }
       // drain: every issued copy must land before the CTA may exit
-      const int64_t first = it > kScanStages ? it - kScanStages : 0;
-      for (int64_t j = first; j < it; ++j) {
-        const int stage = static_cast<int>(j % kScanStages);
-        if (!mbar_wait(&sm.full[stage], static_cast<uint32_t>((j / kScanStages) & 1)))
+      for (int j = max(0, issued - kScanStages); j < issued; ++j) {
+        const int st = j % kScanStages;
+        if (!mbar_wait(&sm.full[st], static_cast<uint32_t>((j / kScanStages) & 1)))
           flag_error(dev_err, CSA2_DEVERR_TIMEOUT);
       }
     }
+    pdl_launch_dependents();
     return;
   }
 
-  // -------------------------------------------------------------------- consumers (8 warps)
+  // ---------------------------------------------------------- consumers (2 groups of 8 warps)
+  // Group gi takes the tiles whose issue index has parity gi; within a tile, warp wg of the
+  // group takes rows 16 wg .. 16 wg + 15.
+  const int gi = warp / kScanGroupWarps, wg = warp % kScanGroupWarps;
   const int g = lane >> 2, c = lane & 3;
   const int mi = lane >> 3;
-  const int a_row = 16 * warp + (lane & 7) + ((mi & 1) << 3);
+  const int a_row = 16 * wg + (lane & 7) + ((mi & 1) << 3);
   int cur_b = -1, nb = 0;
   uint32_t bq0[4], bq1[4];
   float wa = 0.0f, wb = 0.0f;
-  int64_t it = 0;
+  int stage = 0, issued = 0;
+  uint32_t phase = 0;
 
   auto flush = [&](int bseq) {
     consumer_bar();
-    for (int i = tid; i < 2 * kHistBins; i += kScanConsumerWarps * 32) {
-      const uint32_t v = (&sm.hist[0][0])[i];
+    for (int i = tid; i < kHistBins; i += kScanConsumerWarps * 32) {
+      const uint32_t v = sm.hist[i];
       if (v) {
-        atomicAdd(hist_g + static_cast<int64_t>(bseq) * 2 * kHistBins + i, v);
-        (&sm.hist[0][0])[i] = 0u;
+        atomicAdd(hist_g + static_cast<int64_t>(bseq) * kHistBins + i, v);
+        sm.hist[i] = 0u;
       }
     }
     consumer_bar();
   };
 
-  for (int64_t v = v_begin; v < v_end; ++v) {
-    const int b = static_cast<int>(v / tiles_per_seq);
-    const int t = static_cast<int>(v - static_cast<int64_t>(b) * tiles_per_seq);
+  int b = b_first, t = t_first;
+  for (int k = 0; k < n_tiles; ++k) {
     if (b != cur_b) {
       if (cur_b >= 0) flush(cur_b);
       cur_b = b;
@@ -167,7 +189,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       for (int s = 0; s < 4; ++s) {
         bq0[s] = bq1[s] = 0u;
         if (g < HI) {
-          const uint32_t* qrow = reinterpret_cast<const uint32_t*>(iq + (static_cast<int64_t>(b) * HI + g) * DI);
+          const uint32_t* qrow =
+              reinterpret_cast<const uint32_t*>(iq + (static_cast<int64_t>(b) * HI + g) * DI);
           bq0[s] = __ldg(qrow + 8 * s + c);
           bq1[s] = __ldg(qrow + 8 * s + 4 + c);
         }
@@ -175,12 +198,24 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       wa = c < 2 ? __ldg(w + b * HI + 2 * c) : 0.0f;
       wb = c < 2 ? __ldg(w + b * HI + 2 * c + 1) : 0.0f;
     }
-    if (t * kScanTile >= nb) continue;
-    const int stage = static_cast<int>(it % kScanStages);
-    const uint32_t parity = static_cast<uint32_t>((it / kScanStages) & 1);
-    ++it;
+    const int tt = t;
+    if (++t == tiles_per_seq) {
+      t = 0;
+      ++b;
+    }
+    if (tt * kScanTile >= nb) continue;
+    const int my_stage = stage;
+    const uint32_t my_phase = phase;
+    const bool mine = (issued & 1) == gi;
+    ++issued;
+    if (++stage == kScanStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+    if (!mine) continue;
     // every lane waits (acquiring the tile), the warp then takes one decision
-    const bool ok = __all_sync(0xFFFFFFFFu, !*abort && wait_or_abort(&sm.full[stage], parity, abort));
+    const bool ok =
+        __all_sync(0xFFFFFFFFu, !*abort && wait_or_abort(&sm.full[my_stage], my_phase, abort));
     if (!ok) {
       if (lane == 0 && !*abort) flag_error(dev_err, CSA2_DEVERR_TIMEOUT);
       *abort = 1;
@@ -188,7 +223,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     }
 
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const uint32_t tile = smem_u32(sm.tiles[stage]);
+    const uint32_t tile = smem_u32(sm.tiles[my_stage]);
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
       const int chunk = 2 * s + (mi >> 1);
@@ -197,7 +232,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       mma_bf16_16816(acc, a0, a1, a2, a3, bq0[s], bq1[s]);
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.empty[stage]);
+    if (lane == 0) mbar_arrive(&sm.empty[my_stage]);
 
     // scores of rows g and g+8 (lanes c = 0 and 1 hold heads 0,1 and 2,3)
     float s0 = wa * fmaxf(acc[0], 0.0f) + wb * fmaxf(acc[1], 0.0f);
@@ -206,18 +241,12 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
     s0 += 0.0f;  // fold -0 onto +0
     s1 += 0.0f;
-    const int t0 = t * kScanTile + 16 * warp + g, t1 = t0 + 8;
+    const int t0 = tt * kScanTile + 16 * wg + g, t1 = t0 + 8;
     const bool v0 = t0 < nb, v1 = t1 < nb;
     if (c == 0) {
-      float* srow = scores + static_cast<int64_t>(b) * n_cap;
-      if (v0) {
-        srow[t0] = s0;
-        atomicAdd(&sm.hist[0][float_key(s0) >> kHistShift], 1u);
-      }
-      if (v1) {
-        srow[t1] = s1;
-        atomicAdd(&sm.hist[0][float_key(s1) >> kHistShift], 1u);
-      }
+      float* srow = scores + static_cast<int64_t>(cur_b) * n_cap;
+      if (v0) srow[t0] = s0;
+      if (v1) srow[t1] = s1;
     }
     float m0 = v0 ? s0 : -INFINITY, m1 = v1 ? s1 : -INFINITY;
 #pragma unroll
@@ -226,137 +255,284 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       m1 = fmaxf(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, off));
     }
     if (lane == 0) {
-      const int j0 = (t * kScanTile + 16 * warp) / S;
-      float* brow = bmax + static_cast<int64_t>(b) * (n_cap / S);
+      const int j0 = (tt * kScanTile + 16 * wg) / S;
+      float* brow = bmax + static_cast<int64_t>(cur_b) * (n_cap / S);
       if (j0 * S < nb) {
         brow[j0] = m0;
-        atomicAdd(&sm.hist[1][float_key(m0) >> kHistShift], 1u);
+        atomicAdd(&sm.hist[float_key(m0) >> kHistShift], 1u);
       }
       if ((j0 + 1) * S < nb) {
         brow[j0 + 1] = m1;
-        atomicAdd(&sm.hist[1][float_key(m1) >> kHistShift], 1u);
+        atomicAdd(&sm.hist[float_key(m1) >> kHistShift], 1u);
       }
     }
   }
+  pdl_launch_dependents();
   if (cur_b >= 0) flush(cur_b);
 }
 
+// Block candidates: CTA (chunk, b) handles blocks [8192 chunk, 8192 chunk + 8192) of sequence
+// b. Thread t loads its 32 consecutive block maxima at once, keeps those whose key bin is at or
+// above the threshold bin of the max(K, P)-th block, and writes their rank keys in block order
+// into the chunk's region (an exclusive scan over the threads orders them).
 __global__ void __launch_bounds__(kCollectThreads)
-    topk_collect_kernel(const float* __restrict__ scores, const float* __restrict__ bmax,
-                        const int32_t* __restrict__ N, int n_cap, int K, int P,
-                        const uint32_t* __restrict__ hist_g, uint32_t* __restrict__ cnt,
-                        uint64_t* __restrict__ cand) {
+    block_collect_kernel(const float* __restrict__ bmax, const int32_t* __restrict__ N, int n_cap,
+                         int K, int P, const uint32_t* __restrict__ hist_g,
+                         uint32_t* __restrict__ ccnt, uint64_t* __restrict__ cand) {
+  constexpr int kPer = kCollectChunk / kCollectThreads;  // 32 blocks per thread
   __shared__ uint32_t part[kCollectThreads];
-  __shared__ int bin_sh;
-  const int b = blockIdx.y, prob = blockIdx.z;
+  __shared__ uint32_t scan[33];
+  __shared__ int sh[4];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int b = blockIdx.y, chunk = blockIdx.x;
   const int nb = max(0, min(__ldg(N + b), n_cap));
-  const int n_items = prob == 0 ? nb : (nb + S - 1) / S;
-  const int k_take = min(prob == 0 ? K : P, n_items);
-  const int start = blockIdx.x * kCollectChunk;
-  if (k_take == 0 || start >= n_items) return;
-  const int64_t pr = static_cast<int64_t>(b) * 2 + prob;
-  const int T0 = block_find_bin4096(hist_g + pr * kHistBins, static_cast<uint32_t>(k_take), part,
-                                    &bin_sh);
-  const float* src = prob == 0 ? scores + static_cast<int64_t>(b) * n_cap
-                               : bmax + static_cast<int64_t>(b) * (n_cap / S);
-  uint32_t* counter = cnt + pr;
-  uint64_t* out = cand + pr * kCand;
-  const int end = min(start + kCollectChunk, n_items);
-  const int lane = threadIdx.x & 31;
-  for (int i0 = start; i0 < end; i0 += kCollectThreads) {
-    const int i = i0 + threadIdx.x;
-    float v = 0.0f;
-    bool take = false;
-    if (i < end) {
-      v = src[i];
-      take = static_cast<int>(float_key(v) >> kHistShift) >= T0;
+  const int nbl = (nb + S - 1) / S;
+  const int kw = min(max(K, P), nbl);
+  const int start = chunk * kCollectChunk;
+  if (kw == 0 || start >= nbl) return;
+  const int nchunks = (n_cap / S + kCollectChunk - 1) / kCollectChunk;
+  const float* src = bmax + static_cast<int64_t>(b) * (n_cap / S);
+  const int i0 = start + kPer * threadIdx.x;
+  float v[kPer];
+  if (((reinterpret_cast<uintptr_t>(src + i0) & 15u) == 0) && i0 + kPer <= nbl) {
+#pragma unroll
+    for (int m = 0; m < kPer / 4; ++m) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(src + i0) + m);
+      v[4 * m] = f.x;
+      v[4 * m + 1] = f.y;
+      v[4 * m + 2] = f.z;
+      v[4 * m + 3] = f.w;
     }
-    const uint32_t ball = __ballot_sync(0xFFFFFFFFu, take);
-    if (ball == 0) continue;
-    uint32_t base = 0;
-    if (lane == 0) base = atomicAdd(counter, __popc(ball));
-    base = __shfl_sync(0xFFFFFFFFu, base, 0);
-    if (take) {
-      const uint32_t slot = base + __popc(ball & ((1u << lane) - 1u));
-      if (slot < kCand) out[slot] = rank_key(v, static_cast<uint32_t>(i));
+  } else {
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) v[j] = i0 + j < nbl ? __ldg(src + i0 + j) : 0.0f;
+  }
+  const int T0 = block_find_bin4096(hist_g + static_cast<int64_t>(b) * kHistBins,
+                                    static_cast<uint32_t>(kw), part, sh);
+  uint32_t mask = 0, c = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    if (i0 + j < nbl && static_cast<int>(float_key(v[j]) >> kHistShift) >= T0) {
+      mask |= 1u << j;
+      ++c;
     }
   }
+  uint32_t total;
+  uint32_t slot = block_exclusive_scan(c, scan, &total);
+  uint64_t* out = cand + (static_cast<int64_t>(b) * nchunks + chunk) * kCollectChunk;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j)
+    if ((mask >> j) & 1u) out[slot++] = rank_key(v[j], static_cast<uint32_t>(i0 + j));
+  if (threadIdx.x == 0) ccnt[static_cast<int64_t>(b) * nchunks + chunk] = total;
 }
 
 struct FinalSmem {
-  uint64_t cand[kCand];
-  int32_t sel[kMaxSel];
-  uint32_t hist[256];
-  RadixState st;
-  int nsel;
+  union {
+    uint64_t cand[kSmemKeys];        // block candidates (in block order)
+    uint32_t skey[2 * kSmemKeys];    // score keys of the selected blocks' positions
+  } u;
+  int32_t wide[kMaxSel];             // top max(K, P) blocks, ascending
+  uint64_t wide_key[kMaxSel];        // their rank keys
+  union {
+    int32_t chunk_pre[kMaxSel + 1];  // candidate prefix over chunks (while loading candidates)
+    int32_t pos_blk[kMaxSel];        // top-K blocks (hold every Top-K position), ascending
+  } v;
+  uint8_t flag[kMaxSel];             // bit 0: wide[i] is in the pool; bit 1: in the top-K blocks
+  SelectScratch sc;
+};
+
+static_assert(sizeof(FinalSmem) <= 227 * 1024, "index_final_kernel shared memory");
+
+// Rank key of block candidate i, with the chunked layout resolved by a binary search over the
+// chunk prefix (only used when the candidates do not fit in shared memory).
+struct ChunkedKeys {
+  const uint64_t* base;
+  const int32_t* pre;
+  int nchunks;
+  __device__ uint64_t operator()(int i) const {
+    int lo = 0, hi = nchunks - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= i) lo = mid;
+      else hi = mid - 1;
+    }
+    return base[static_cast<int64_t>(lo) * kCollectChunk + (i - pre[lo])];
+  }
 };
 
 __global__ void __launch_bounds__(kFinalThreads)
-    topk_final_kernel(const float* __restrict__ scores, const float* __restrict__ bmax,
-                      const int32_t* __restrict__ N, int n_cap, int K, int P,
-                      const uint32_t* __restrict__ cnt, const uint64_t* __restrict__ cand,
-                      int32_t* __restrict__ topk, int32_t* __restrict__ pool) {
+    index_final_kernel(const float* __restrict__ scores, const int32_t* __restrict__ N, int n_cap,
+                       int K, int P, const uint32_t* __restrict__ ccnt,
+                       const uint64_t* __restrict__ cand, int32_t* __restrict__ topk,
+                       int32_t* __restrict__ pool) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   FinalSmem& sm = *reinterpret_cast<FinalSmem*>(smem_raw);
-  const int b = blockIdx.x, prob = blockIdx.y, tid = threadIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int b = blockIdx.x, tid = threadIdx.x;
   const int nb = max(0, min(__ldg(N + b), n_cap));
-  const int n_items = prob == 0 ? nb : (nb + S - 1) / S;
-  const int kk = prob == 0 ? K : P;
-  const int k_take = min(kk, n_items);
-  const int64_t pr = static_cast<int64_t>(b) * 2 + prob;
-  const uint32_t count = cnt[pr];
-  if (tid == 0) sm.nsel = 0;
+  const int nbl = (nb + S - 1) / S;
+  const int kw = min(max(K, P), nbl);  // blocks that hold every Top-K position and the pool
+  const int kp = min(P, nbl);
+  const int kk = min(K, nb);
+  const int nchunks = (n_cap / S + kCollectChunk - 1) / kCollectChunk;
+  const int nch = (nbl + kCollectChunk - 1) / kCollectChunk;
+  int32_t* pool_out = pool + static_cast<int64_t>(b) * P * S;
+  int32_t* topk_out = topk + static_cast<int64_t>(b) * K;
+  if (kw == 0) {
+    for (int i = tid; i < P * S; i += kFinalThreads) pool_out[i] = -1;
+    for (int i = tid; i < K; i += kFinalThreads) topk_out[i] = -1;
+    return;
+  }
 
-  if (k_take > 0 && count <= static_cast<uint32_t>(kCand)) {
-    const uint64_t* src = cand + pr * kCand;
-    for (int i = tid; i < static_cast<int>(count); i += kFinalThreads) sm.cand[i] = src[i];
-    __syncthreads();
-    const uint64_t* c = sm.cand;
-    auto get = [c](int i) { return c[i]; };
-    block_radix_select(get, static_cast<int>(count), static_cast<uint32_t>(k_take), sm.hist, &sm.st);
-    const RadixState st = sm.st;
-    for (int i = tid; i < static_cast<int>(count); i += kFinalThreads) {
-      const uint64_t key = c[i];
-      if (radix_selected(key, st)) {
-        const int slot = atomicAdd(&sm.nsel, 1);
-        if (slot < kMaxSel) sm.sel[slot] = static_cast<int32_t>(rank_key_index(key));
-      }
+  // ---- block candidates in block order
+  const uint32_t* cnts = ccnt + static_cast<int64_t>(b) * nchunks;
+  const uint64_t* cbase = cand + static_cast<int64_t>(b) * nchunks * kCollectChunk;
+  // prefix over chunk counts (thread c owns chunks 4c..4c+3)
+  {
+    uint32_t cv[4];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = 4 * tid + j;
+      cv[j] = c < nch ? __ldg(cnts + c) : 0u;
+      sum += cv[j];
     }
-  } else if (k_take > 0) {
-    // candidate overflow (many near-equal scores): exact select over the whole array
-    const float* arr = prob == 0 ? scores + static_cast<int64_t>(b) * n_cap
-                                 : bmax + static_cast<int64_t>(b) * (n_cap / S);
-    auto get = [arr](int i) { return rank_key(arr[i], static_cast<uint32_t>(i)); };
+    uint32_t total;
+    uint32_t run = block_exclusive_scan(sum, sm.sc.scan, &total);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = 4 * tid + j;
+      if (c < nch) sm.v.chunk_pre[c] = static_cast<int32_t>(run);
+      run += cv[j];
+    }
+    if (tid == 0) sm.v.chunk_pre[nch] = static_cast<int32_t>(total);
+  }
+  __syncthreads();
+  const int C = sm.v.chunk_pre[nch];
+  const bool in_smem = C <= kSmemKeys;
+  if (in_smem) {
+    // copy chunk regions into one ordered array (independent loads, 8 per round)
+    for (int base = 0; base < C; base += 8 * kFinalThreads) {
+      uint64_t vals[8];
+      int dst[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = base + j * kFinalThreads + tid;
+        dst[j] = -1;
+        if (i < C) {
+          int lo = 0, hi = nch - 1;
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (sm.v.chunk_pre[mid] <= i) lo = mid;
+            else hi = mid - 1;
+          }
+          vals[j] = __ldg(cbase + static_cast<int64_t>(lo) * kCollectChunk + (i - sm.v.chunk_pre[lo]));
+          dst[j] = i;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (dst[j] >= 0) sm.u.cand[dst[j]] = vals[j];
+    }
     __syncthreads();
-    block_radix_select(get, n_items, static_cast<uint32_t>(k_take), sm.hist, &sm.st);
-    const RadixState st = sm.st;
-    for (int i = tid; i < n_items; i += kFinalThreads) {
-      if (radix_selected(get(i), st)) {
-        const int slot = atomicAdd(&sm.nsel, 1);
-        if (slot < kMaxSel) sm.sel[slot] = i;
+  }
+  const ChunkedKeys gk{cbase, sm.v.chunk_pre, nch};
+  const uint64_t* sk = sm.u.cand;
+  auto cand_key = [&](int i) -> uint64_t { return in_smem ? sk[i] : gk(i); };
+
+  // ---- top kw blocks, ascending
+  block_radix_select(cand_key, C, static_cast<uint32_t>(kw), sm.sc);
+  {
+    const RadixState st = sm.sc.st;
+    block_ordered_compact(
+        C, [&](int i) { return radix_selected(cand_key(i), st); },
+        [&](int i, uint32_t slot) {
+          if (slot < kMaxSel) {
+            const uint64_t key = cand_key(i);
+            sm.wide[slot] = static_cast<int32_t>(rank_key_index(key));
+            sm.wide_key[slot] = key;
+          }
+        },
+        sm.sc.scan);
+  }
+  for (int i = tid; i < kw; i += kFinalThreads) sm.flag[i] = 3;
+  __syncthreads();
+
+  // ---- the pool (top kp blocks) and the position blocks (top kkb blocks) are the top parts of
+  // the wide set; the smaller of the two is selected again among the wide keys
+  const int kkb = min(K, nbl);
+  const uint64_t* wk = sm.wide_key;
+  auto wide_key = [wk](int i) { return wk[i]; };
+  if (kp < kw || kkb < kw) {
+    const int ksub = kp < kw ? kp : kkb;
+    const uint8_t clear = kp < kw ? 1 : 2;
+    block_radix_select(wide_key, kw, static_cast<uint32_t>(ksub), sm.sc);
+    const RadixState st = sm.sc.st;
+    for (int i = tid; i < kw; i += kFinalThreads)
+      if (!radix_selected(wk[i], st)) sm.flag[i] &= static_cast<uint8_t>(~clear);
+    __syncthreads();
+  }
+  {
+    const uint32_t n_pool = block_ordered_compact(
+        kw, [&](int i) { return (sm.flag[i] & 1) != 0; },
+        [&](int i, uint32_t slot) {
+          for (int r = 0; r < S; ++r) {
+            const int p = sm.wide[i] * S + r;
+            pool_out[slot * S + r] = p < nb ? p : -1;
+          }
+        },
+        sm.sc.scan);
+    for (int i = static_cast<int>(n_pool) * S + tid; i < P * S; i += kFinalThreads)
+      pool_out[i] = -1;
+    block_ordered_compact(
+        kw, [&](int i) { return (sm.flag[i] & 2) != 0; },
+        [&](int i, uint32_t slot) { sm.v.pos_blk[slot] = sm.wide[i]; }, sm.sc.scan);
+  }
+  __syncthreads();
+
+  // ---- position Top-K over the top-K blocks' positions (slot order = ascending position)
+  const int L = kkb * S;
+  const float* srow = scores + static_cast<int64_t>(b) * n_cap;
+  const bool keys64 = L <= kSmemKeys;
+  for (int base = 0; base < L; base += 8 * kFinalThreads) {
+    float vals[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = base + j * kFinalThreads + tid;
+      const int p = i < L ? sm.v.pos_blk[i / S] * S + (i % S) : nb;
+      vals[j] = p < nb ? __ldg(srow + p) : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = base + j * kFinalThreads + tid;
+      if (i < L) {
+        const uint32_t p = static_cast<uint32_t>(sm.v.pos_blk[i / S] * S + (i % S));
+        const bool valid = p < static_cast<uint32_t>(nb);
+        if (keys64) sm.u.cand[i] = valid ? rank_key(vals[j], p) : 0ull;
+        else sm.u.skey[i] = valid ? float_key(vals[j]) : 0u;
       }
     }
   }
   __syncthreads();
-  int n2 = 1;
-  while (n2 < k_take) n2 <<= 1;
-  for (int i = k_take + tid; i < n2; i += kFinalThreads) sm.sel[i] = 0x7FFFFFFF;
-  __syncthreads();
-  if (k_take > 1) block_bitonic_sort_i32(sm.sel, n2);
-  if (prob == 0) {
-    int32_t* dst = topk + static_cast<int64_t>(b) * K;
-    for (int i = tid; i < K; i += kFinalThreads) dst[i] = i < k_take ? sm.sel[i] : -1;
-  } else {
-    int32_t* dst = pool + static_cast<int64_t>(b) * P * S;
-    for (int i = tid; i < P * S; i += kFinalThreads) {
-      const int j = i / S, r = i % S;
-      int v = -1;
-      if (j < k_take) {
-        const int p = sm.sel[j] * S + r;
-        v = p < nb ? p : -1;
-      }
-      dst[i] = v;
-    }
+  auto pos_key = [&](int i) -> uint64_t {
+    if (keys64) return sm.u.cand[i];
+    const uint32_t hk = sm.u.skey[i];
+    if (hk == 0u) return 0ull;  // a position past N: below every real key
+    const uint32_t p = static_cast<uint32_t>(sm.v.pos_blk[i / S] * S + (i % S));
+    return (static_cast<uint64_t>(hk) << 32) | static_cast<uint64_t>(~p);
+  };
+  block_radix_select(pos_key, L, static_cast<uint32_t>(kk), sm.sc);
+  {
+    const RadixState st = sm.sc.st;
+    const uint32_t n_sel = block_ordered_compact(
+        L, [&](int i) { const uint64_t k = pos_key(i); return k != 0ull && radix_selected(k, st); },
+        [&](int i, uint32_t slot) {
+          if (slot < static_cast<uint32_t>(K)) topk_out[slot] = sm.v.pos_blk[i / S] * S + (i % S);
+        },
+        sm.sc.scan);
+    for (int i = static_cast<int>(n_sel) + tid; i < K; i += kFinalThreads) topk_out[i] = -1;
   }
 }
 
@@ -367,48 +543,57 @@ constexpr int kReThreads = 256;
 
 // 8 lanes per pool slot, 8 dims (16 bytes of key) per lane; writes the slot's rank key (0 for an
 // empty or out-of-range slot, which is below every real key).
-__global__ void __launch_bounds__(kReThreads)
+__global__ void __launch_bounds__(kReThreads, 3)
     reindex_score_kernel(const uint16_t* __restrict__ iq, const float* __restrict__ w,
                          const uint16_t* __restrict__ ik_cache, const int32_t* __restrict__ N,
                          int n_cap, const int32_t* __restrict__ pool, int L,
                          uint64_t* __restrict__ keys, int32_t* dev_err) {
+  __shared__ float qs[HI][DI];
+  __shared__ float wh[HI];
+  pdl_wait();
+  pdl_launch_dependents();
   const int b = blockIdx.y;
   const int lane = threadIdx.x & 31, sub = lane & 7;
   const int nb = clamp_len(N, b, n_cap, threadIdx.x == 0 && blockIdx.x == 0 ? dev_err : nullptr);
-  float qv[HI][8];
-#pragma unroll
-  for (int h = 0; h < HI; ++h) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(iq + (static_cast<int64_t>(b) * HI + h) * DI) + sub);
-    const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      qv[h][2 * k] = bf16lo(uw[k]);
-      qv[h][2 * k + 1] = bf16hi(uw[k]);
-    }
+  {
+    const int h = threadIdx.x >> 6, i = threadIdx.x & 63;  // 256 threads = 4 heads x 64 dims
+    const uint16_t qb = iq[(static_cast<int64_t>(b) * HI + h) * DI + i];
+    qs[h][i] = __uint_as_float(static_cast<uint32_t>(qb) << 16);
+    if (threadIdx.x < HI) wh[threadIdx.x] = __ldg(w + b * HI + threadIdx.x);
   }
-  float wh[HI];
-#pragma unroll
-  for (int h = 0; h < HI; ++h) wh[h] = __ldg(w + b * HI + h);
+  __syncthreads();
   const int slot0 = blockIdx.x * kReSlotsPerCta;
   const int slot_end = min(slot0 + kReSlotsPerCta, L);
   constexpr int per_iter = kReThreads / 8;
-  // the trip count is the same for every thread of the CTA (shuffles below need whole warps)
-  for (int s0 = slot0; s0 < slot_end; s0 += per_iter) {
-    const int s = s0 + (threadIdx.x >> 3);
-    const bool in_range = s < slot_end;
-    const int pos = in_range ? __ldg(pool + static_cast<int64_t>(b) * L + s) : -1;
-    const bool valid = pos >= 0 && pos < nb;
-    if (!valid && pos != -1 && sub == 0) flag_error(dev_err, CSA2_DEVERR_INDEX_RANGE);
+  constexpr int kIter = kReSlotsPerCta / per_iter;
+  // all pool loads, then all key loads, then the arithmetic (two memory round trips per CTA)
+  int pos[kIter];
+#pragma unroll
+  for (int it = 0; it < kIter; ++it) {
+    const int s = slot0 + it * per_iter + (threadIdx.x >> 3);
+    pos[it] = s < slot_end ? __ldg(pool + static_cast<int64_t>(b) * L + s) : -1;
+  }
+  uint4 u[kIter];
+#pragma unroll
+  for (int it = 0; it < kIter; ++it) {
+    const bool valid = pos[it] >= 0 && pos[it] < nb;
+    if (!valid && pos[it] != -1 && sub == 0) flag_error(dev_err, CSA2_DEVERR_INDEX_RANGE);
+    u[it] = valid ? ldg_nc_v4(reinterpret_cast<const uint4*>(
+                        ik_cache + (static_cast<int64_t>(b) * n_cap + pos[it]) * DI) + sub)
+                  : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int it = 0; it < kIter; ++it) {
+    const int s = slot0 + it * per_iter + (threadIdx.x >> 3);
+    const bool valid = pos[it] >= 0 && pos[it] < nb;
+    const uint32_t uw[4] = {u[it].x, u[it].y, u[it].z, u[it].w};
     float d[HI] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (valid) {
-      const uint4 u = ldg_nc_v4(reinterpret_cast<const uint4*>(ik_cache + (static_cast<int64_t>(b) * n_cap + pos) * DI) + sub);
-      const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float x0 = bf16lo(uw[k]), x1 = bf16hi(uw[k]);
+    for (int k = 0; k < 4; ++k) {
+      const float x0 = bf16lo(uw[k]), x1 = bf16hi(uw[k]);
 #pragma unroll
-        for (int h = 0; h < HI; ++h) d[h] = fmaf(qv[h][2 * k + 1], x1, fmaf(qv[h][2 * k], x0, d[h]));
-      }
+      for (int h = 0; h < HI; ++h)
+        d[h] = fmaf(qs[h][8 * sub + 2 * k + 1], x1, fmaf(qs[h][8 * sub + 2 * k], x0, d[h]));
     }
 #pragma unroll
     for (int h = 0; h < HI; ++h) {
@@ -416,66 +601,107 @@ __global__ void __launch_bounds__(kReThreads)
       d[h] += __shfl_xor_sync(0xFFFFFFFFu, d[h], 2);
       d[h] += __shfl_xor_sync(0xFFFFFFFFu, d[h], 4);
     }
-    if (sub == 0 && in_range) {
+    if (sub == 0 && s < slot_end) {
       float score = 0.0f;
 #pragma unroll
       for (int h = 0; h < HI; ++h) score = fmaf(wh[h], fmaxf(d[h], 0.0f), score);
-      keys[static_cast<int64_t>(b) * L + s] = valid ? rank_key(score, static_cast<uint32_t>(pos)) : 0ull;
+      keys[static_cast<int64_t>(b) * L + s] =
+          valid ? rank_key(score, static_cast<uint32_t>(pos[it])) : 0ull;
     }
   }
 }
 
+constexpr int kReCand = 4096;  // reindex candidates at or above the threshold bin
+
 struct ReFinalSmem {
-  uint64_t keys[kCand];
+  uint64_t keys[kSmemKeys];
+  uint64_t cand[kReCand];
   int32_t sel[kMaxSel];
-  uint32_t hist[256];
-  RadixState st;
-  int nsel;
+  SelectScratch sc;
   int nvalid;
+  int unsorted;
 };
 
+static_assert(sizeof(ReFinalSmem) <= 227 * 1024, "reindex_final_kernel shared memory");
+
+// One CTA per sequence: the Top-K of the pool's rank keys (0 = empty slot). The key load also
+// histograms the top 12 bits of every real key; only the keys at or above the bin that holds the
+// K-th key enter the radix select (unless more than kReCand do). Winners come out in pool order,
+// which is ascending position for a pool built by the Full-mode indexer; any other pool order is
+// sorted afterwards.
 __global__ void __launch_bounds__(kFinalThreads)
     reindex_final_kernel(const uint64_t* __restrict__ keys_g, int L, int K,
                          int32_t* __restrict__ topk) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   ReFinalSmem& sm = *reinterpret_cast<ReFinalSmem*>(smem_raw);
+  pdl_wait();
+  pdl_launch_dependents();
   const int b = blockIdx.x, tid = threadIdx.x;
   const uint64_t* src = keys_g + static_cast<int64_t>(b) * L;
-  const bool in_smem = L <= kCand;
+  const bool in_smem = L <= kSmemKeys;
+  for (int i = tid; i < kDigitBins; i += kFinalThreads) sm.sc.hist[i] = 0u;
   if (tid == 0) {
-    sm.nsel = 0;
     sm.nvalid = 0;
+    sm.unsorted = 0;
   }
   __syncthreads();
   int nv = 0;
-  for (int i = tid; i < L; i += kFinalThreads) {
-    const uint64_t k = src[i];
-    if (in_smem) sm.keys[i] = k;
-    nv += k != 0ull;
+  for (int base = 0; base < L; base += 8 * kFinalThreads) {
+    uint64_t v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = base + j * kFinalThreads + tid;
+      v[j] = i < L ? __ldg(src + i) : 0ull;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = base + j * kFinalThreads + tid;
+      if (i < L) {
+        if (in_smem) sm.keys[i] = v[j];
+        if (v[j] != 0ull) {
+          ++nv;
+          atomicAdd(&sm.sc.hist[static_cast<uint32_t>(v[j] >> 52)], 1u);
+        }
+      }
+    }
   }
   nv = __reduce_add_sync(0xFFFFFFFFu, nv);
   if ((tid & 31) == 0) atomicAdd(&sm.nvalid, nv);
   __syncthreads();
   const int k_take = min(K, sm.nvalid);
   const uint64_t* c = in_smem ? sm.keys : src;
-  auto get = [c](int i) { return c[i]; };
-  block_radix_select(get, L, static_cast<uint32_t>(k_take), sm.hist, &sm.st);
-  const RadixState st = sm.st;
   if (k_take > 0) {
-    for (int i = tid; i < L; i += kFinalThreads) {
-      const uint64_t key = c[i];
-      if (key != 0ull && radix_selected(key, st)) {
-        const int slot = atomicAdd(&sm.nsel, 1);
-        if (slot < kMaxSel) sm.sel[slot] = static_cast<int32_t>(rank_key_index(key));
-      }
+    const int T0 = block_find_bin4096(sm.sc.hist, static_cast<uint32_t>(k_take), sm.sc.part,
+                                      sm.sc.ints);
+    const uint32_t n_cand = block_ordered_compact(
+        L, [&](int i) { const uint64_t k = c[i]; return k != 0ull && static_cast<int>(k >> 52) >= T0; },
+        [&](int i, uint32_t slot) { if (slot < kReCand) sm.cand[slot] = c[i]; }, sm.sc.scan);
+    __syncthreads();
+    const bool small = n_cand <= static_cast<uint32_t>(kReCand);
+    const uint64_t* kk = small ? sm.cand : c;
+    const int nk = small ? static_cast<int>(n_cand) : L;
+    auto get = [kk](int i) { return kk[i]; };
+    block_radix_select(get, nk, static_cast<uint32_t>(k_take), sm.sc);
+    const RadixState st = sm.sc.st;
+    block_ordered_compact(
+        nk, [&](int i) { const uint64_t k = kk[i]; return k != 0ull && radix_selected(k, st); },
+        [&](int i, uint32_t slot) {
+          if (slot < kMaxSel) sm.sel[slot] = static_cast<int32_t>(rank_key_index(kk[i]));
+        },
+        sm.sc.scan);
+    __syncthreads();
+    for (int i = tid; i + 1 < k_take; i += kFinalThreads)
+      if (sm.sel[i] >= sm.sel[i + 1]) sm.unsorted = 1;
+    __syncthreads();
+    if (sm.unsorted) {
+      int n2 = 1;
+      while (n2 < k_take) n2 <<= 1;
+      for (int i = k_take + tid; i < n2; i += kFinalThreads) sm.sel[i] = 0x7FFFFFFF;
+      __syncthreads();
+      block_bitonic_sort_i32(sm.sel, n2);
     }
   }
   __syncthreads();
-  int n2 = 1;
-  while (n2 < k_take) n2 <<= 1;
-  for (int i = k_take + tid; i < n2; i += kFinalThreads) sm.sel[i] = 0x7FFFFFFF;
-  __syncthreads();
-  if (k_take > 1) block_bitonic_sort_i32(sm.sel, n2);
   int32_t* dst = topk + static_cast<int64_t>(b) * K;
   for (int i = tid; i < K; i += kFinalThreads) dst[i] = i < k_take ? sm.sel[i] : -1;
 }
@@ -485,25 +711,25 @@ __global__ void __launch_bounds__(kFinalThreads)
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct FullLayout {
-  size_t scores, bmax, hist, cnt, cand, total, zero_begin, zero_bytes;
+  size_t scores, bmax, hist, ccnt, cand, total;
+  int nchunks;
 };
 
 FullLayout full_layout(int B, int n_cap) {
   FullLayout l;
+  l.nchunks = (n_cap / S + kCollectChunk - 1) / kCollectChunk;
   size_t off = 0;
   l.scores = off;
   off = align256(off + static_cast<size_t>(B) * n_cap * sizeof(float));
   l.bmax = off;
   off = align256(off + static_cast<size_t>(B) * (n_cap / S) * sizeof(float));
   l.hist = off;
-  off += static_cast<size_t>(B) * 2 * kHistBins * sizeof(uint32_t);
-  l.cnt = off;
-  off = align256(off + static_cast<size_t>(B) * 2 * sizeof(uint32_t));
+  off = align256(off + static_cast<size_t>(B) * kHistBins * sizeof(uint32_t));
+  l.ccnt = off;
+  off = align256(off + static_cast<size_t>(B) * l.nchunks * sizeof(uint32_t));
   l.cand = off;
-  off = align256(off + static_cast<size_t>(B) * 2 * kCand * sizeof(uint64_t));
+  off = align256(off + static_cast<size_t>(B) * l.nchunks * kCollectChunk * sizeof(uint64_t));
   l.total = off;
-  l.zero_begin = l.hist;
-  l.zero_bytes = l.cand - l.hist;
   return l;
 }
 
@@ -557,7 +783,7 @@ cudaError_t launch_index_full(const void* iq, const float* w, const void* ik_cac
   float* scores = reinterpret_cast<float*>(base + l.scores);
   float* bmax = reinterpret_cast<float*>(base + l.bmax);
   uint32_t* hist = reinterpret_cast<uint32_t*>(base + l.hist);
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(base + l.cnt);
+  uint32_t* ccnt = reinterpret_cast<uint32_t*>(base + l.ccnt);
   uint64_t* cand = reinterpret_cast<uint64_t*>(base + l.cand);
 
   EncodeTiledFn enc = encode_fn();
@@ -579,11 +805,12 @@ cudaError_t launch_index_full(const void* iq, const float* w, const void* ik_cac
     std::lock_guard<std::mutex> lock(g_attr_mu);
     cudaError_t e = set_smem(index_scan_kernel, sizeof(ScanSmem), done_scan);
     if (e != cudaSuccess) return e;
-    e = set_smem(topk_final_kernel, sizeof(FinalSmem), done_final);
+    e = set_smem(index_final_kernel, sizeof(FinalSmem), done_final);
     if (e != cudaSuccess) return e;
   }
 
-  cudaError_t e = cudaMemsetAsync(base + l.zero_begin, 0, l.zero_bytes, s);
+  // the block histogram accumulates across the scan's CTAs: zero it first
+  cudaError_t e = cudaMemsetAsync(hist, 0, static_cast<size_t>(B) * kHistBins * sizeof(uint32_t), s);
   if (e != cudaSuccess) return e;
   const int64_t tiles = static_cast<int64_t>(B) * ((n_cap + kScanTile - 1) / kScanTile);
   const int grid = static_cast<int>(std::min<int64_t>(device_sm_count(), tiles));
@@ -594,17 +821,18 @@ cudaError_t launch_index_full(const void* iq, const float* w, const void* ik_cac
   count_launches(1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   profile_begin(CSA2_KERNEL_INDEX_SELECT, s);
-  const dim3 cgrid((n_cap + kCollectChunk - 1) / kCollectChunk, B, 2);
-  topk_collect_kernel<<<cgrid, kCollectThreads, 0, s>>>(scores, bmax, N, n_cap, K, P, hist, cnt,
-                                                         cand);
+  e = launch_pdl(block_collect_kernel, dim3(l.nchunks, B), dim3(kCollectThreads), 0, s,
+                 static_cast<const float*>(bmax), N, n_cap, K, P,
+                 static_cast<const uint32_t*>(hist), ccnt, cand);
   count_launches(1);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  topk_final_kernel<<<dim3(B, 2), kFinalThreads, sizeof(FinalSmem), s>>>(scores, bmax, N, n_cap,
-                                                                          K, P, cnt, cand, topk,
-                                                                          pool);
+  if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
+  e = launch_pdl(index_final_kernel, dim3(B), dim3(kFinalThreads), sizeof(FinalSmem), s,
+                 static_cast<const float*>(scores), N, n_cap, K, P,
+                 static_cast<const uint32_t*>(ccnt), static_cast<const uint64_t*>(cand), topk,
+                 pool);
   profile_end(CSA2_KERNEL_INDEX_SELECT, s);
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 size_t index_reindex_workspace_bytes(int B, int L, int K) {
@@ -625,16 +853,17 @@ cudaError_t launch_index_reindex(const void* iq, const float* w, const void* ik_
   }
   const dim3 grid((L + kReSlotsPerCta - 1) / kReSlotsPerCta, B);
   profile_begin(CSA2_KERNEL_REINDEX, s);
-  reindex_score_kernel<<<grid, kReThreads, 0, s>>>(static_cast<const uint16_t*>(iq), w,
-                                                   static_cast<const uint16_t*>(ik_cache), N,
-                                                   n_cap, pool, L, keys, dev_err);
+  cudaError_t e = launch_pdl(reindex_score_kernel, grid, dim3(kReThreads), 0, s,
+                             static_cast<const uint16_t*>(iq), w,
+                             static_cast<const uint16_t*>(ik_cache), N, n_cap, pool, L, keys,
+                             dev_err);
   count_launches(1);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  reindex_final_kernel<<<B, kFinalThreads, sizeof(ReFinalSmem), s>>>(keys, L, K, topk);
+  if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
+  e = launch_pdl(reindex_final_kernel, dim3(B), dim3(kFinalThreads), sizeof(ReFinalSmem), s,
+                 static_cast<const uint64_t*>(keys), L, K, topk);
   profile_end(CSA2_KERNEL_REINDEX, s);
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace csa2

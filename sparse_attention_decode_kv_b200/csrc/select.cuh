@@ -1,68 +1,77 @@
-// select.cuh -- exact Top-K selection helpers used by the indexer kernels.
+// select.cuh -- exact Top-K selection primitives used by the indexer kernels.
 //
 // Ranking: "DeepSeek V4.1 Flash 拆解" (austincafe.tech), section 一, selects a Top-K of indexer
-// scores (and a Top-2048 of blocks); ties go to the lower index. Every candidate carries a 64-bit
+// scores (and a Top-2048 of blocks); ties go to the lower index. Every item carries a 64-bit
 // rank key (monotone score key in the high word, inverted index in the low word), so the Top-K is
 // the set of the k largest keys, which are all distinct. The selection is an MSB-first radix
-// select over 8-bit digits of that key: each pass histograms the next digit of the keys that
-// still match the known prefix, and stops as soon as the bin holding the k-th key is taken whole.
+// select: one min/max pass finds the bits all keys share, then each pass histograms the next 12
+// bits of the keys that still match the known prefix (4096 shared-memory bins) and stops as soon
+// as the bin holding the k-th key is taken whole. Winners are emitted in item order by an
+// order-preserving compaction, so item order (ascending index) needs no sort.
 #pragma once
 
 #include "common.cuh"
 
 namespace csa2 {
 
-constexpr int kHistBins = 4096;   // first-level histogram: top 12 bits of the 32-bit score key
+constexpr int kHistBins = 4096;   // first-level histogram of the scan: top 12 bits of the key
 constexpr int kHistShift = 20;
+constexpr int kDigitBits = 12;    // radix digit of the in-CTA select
+constexpr int kDigitBins = 1 << kDigitBits;
 
-// One warp finds, in a 256-bin histogram, the largest digit d with sum_{d' >= d} h[d'] >= need.
-// Returns d; *above = sum_{d' > d} h[d'].
-__device__ __forceinline__ int warp_find_digit256(const uint32_t* h, uint32_t need,
-                                                  uint32_t* above) {
-  const int lane = threadIdx.x & 31;
-  uint32_t q = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) q += h[8 * lane + i];
-  uint32_t suf = q;  // inclusive suffix sum over lanes >= lane
+// ------------------------------------------------------------------------------- block scans
+
+// Exclusive prefix sum of one value per thread over the CTA; *total receives the sum.
+// scratch: 33 shared words. Must be called by every thread of the CTA.
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* scratch,
+                                                         uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  uint32_t incl = v;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
-    const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, suf, off);
-    if (lane + off < 32) suf += v;
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += y;
   }
-  const uint32_t ball = __ballot_sync(0xFFFFFFFFu, suf >= need);
-  const int L = ball ? 31 - __clz(ball) : 0;
-  uint32_t run = __shfl_sync(0xFFFFFFFFu, suf, (L + 1) & 31);
-  if (L == 31) run = 0;
-  int d = 8 * L;
-  if (lane == L) {
-    for (int i = 7; i >= 0; --i) {
-      const uint32_t c = h[8 * L + i];
-      if (run + c >= need) {
-        d = 8 * L + i;
-        break;
-      }
-      run += c;
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t wv = lane < nw ? scratch[lane] : 0u;
+    uint32_t wi = wv;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, wi, off);
+      if (lane >= off) wi += y;
     }
+    if (lane < nw) scratch[lane] = wi - wv;  // exclusive warp offsets
+    if (lane == 31) scratch[32] = wi;
   }
-  d = __shfl_sync(0xFFFFFFFFu, d, L);
-  run = __shfl_sync(0xFFFFFFFFu, run, L);
-  *above = run;
-  return d;
+  __syncthreads();
+  const uint32_t r = scratch[warp] + incl - v;
+  *total = scratch[32];
+  __syncthreads();  // scratch may be reused by the caller
+  return r;
 }
 
-// The whole CTA finds the first-level threshold bin in a kHistBins histogram (global memory):
-// the largest bin T with sum_{bins >= T} >= need. part must hold blockDim.x entries.
+// ------------------------------------------------------------------------------ threshold bin
+
+// The largest bin T of a 4096-bin histogram with sum_{bins >= T} >= need (whole CTA; blockDim.x
+// divides 4096 and is at least 256). `hist` may live in global or shared memory. Every thread
+// loads its contiguous bins at once; the owners of the crossing group resolve the exact bin.
+// shared_int[3] receives the count in the bins above T.
 __device__ __forceinline__ int block_find_bin4096(const uint32_t* hist, uint32_t need,
-                                                  uint32_t* part, int* result) {
+                                                  uint32_t* part, int* shared_int) {
   const int tid = threadIdx.x, nt = blockDim.x;
-  const int per = kHistBins / nt;  // blockDim.x divides 4096
+  const int per = kHistBins / nt;  // 4 (1024 threads) or 16 (256 threads)
+  uint32_t h[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) h[i] = i < per ? hist[tid * per + i] : 0u;
   uint32_t s = 0;
-  for (int i = 0; i < per; ++i) s += hist[tid * per + i];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) s += h[i];
   part[tid] = s;
   __syncthreads();
   if (tid < 32) {
-    // level 1: lanes own nt/32 parts each
-    const int pl = nt / 32;
+    const int pl = nt / 32;  // parts per lane
     uint32_t q = 0;
     for (int i = 0; i < pl; ++i) q += part[tid * pl + i];
     uint32_t suf = q;
@@ -75,27 +84,44 @@ __device__ __forceinline__ int block_find_bin4096(const uint32_t* hist, uint32_t
     const int L = ball ? 31 - __clz(ball) : 0;
     uint32_t run = __shfl_sync(0xFFFFFFFFu, suf, (L + 1) & 31);
     if (L == 31) run = 0;
-    // level 2: walk lane L's parts from the top, then that part's bins
-    int bin = 0;
+    // lane L's parts, resolved by the whole warp (at most 32 parts per lane)
+    const uint32_t pv = tid < pl ? part[L * pl + tid] : 0u;
+    uint32_t psuf = pv;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, psuf, off);
+      if (tid + off < 32) psuf += v;
+    }
+    const uint32_t pball = __ballot_sync(0xFFFFFFFFu, tid < pl && run + psuf >= need);
+    const int j = pball ? 31 - __clz(pball) : 0;
+    const uint32_t above = __shfl_sync(0xFFFFFFFFu, psuf - pv, j);
     if (tid == 0) {
-      int p = L * pl + pl - 1;
-      for (; p > L * pl; --p) {
-        if (run + part[p] >= need) break;
-        run += part[p];
-      }
-      int i = p * per + per - 1;
-      for (; i > p * per; --i) {
-        const uint32_t c = hist[i];
-        if (run + c >= need) break;
-        run += c;
-      }
-      bin = i;
-      *result = bin;
+      shared_int[0] = L * pl + j;
+      shared_int[1] = static_cast<int>(run + above);  // count in the parts above that part
     }
   }
   __syncthreads();
-  return *result;
+  if (tid == shared_int[0]) {
+    uint32_t run = static_cast<uint32_t>(shared_int[1]);
+    int bin = tid * per;
+#pragma unroll
+    for (int i = 15; i >= 0; --i) {
+      if (i >= per) continue;
+      if (run + h[i] >= need) {
+        bin = tid * per + i;
+        break;
+      }
+      run += h[i];
+    }
+    shared_int[2] = bin;
+    shared_int[3] = static_cast<int>(run);
+  }
+  __syncthreads();
+  const int r = shared_int[2];
+  return r;
 }
+
+// ------------------------------------------------------------------------------ radix select
 
 struct RadixState {
   uint64_t prefix;
@@ -104,42 +130,78 @@ struct RadixState {
   int done;
 };
 
-// Top-k of n distinct 64-bit keys by MSB-first radix select (whole CTA). get(i) returns key i.
-// On return st->prefix / st->bits describe the threshold: key i is selected iff its top `bits`
-// bits are >= those of prefix. k must be <= n. hist256: 256 shared words.
+struct SelectScratch {
+  uint32_t hist[kDigitBins];
+  uint32_t part[1024];
+  uint32_t scan[33];
+  int ints[4];
+  uint64_t red_min[32], red_max[32];
+  RadixState st;
+};
+
+// Top-k of n distinct 64-bit keys (whole CTA). get(i) returns key i. On return sc.st describes
+// the threshold: key i is selected iff its top `bits` bits are >= those of prefix. Requires
+// 1 <= k <= n.
 template <class Get>
-__device__ void block_radix_select(const Get& get, int n, uint32_t k, uint32_t* hist256,
-                                   RadixState* st) {
-  const int tid = threadIdx.x, nt = blockDim.x;
-  if (tid == 0) {
-    st->prefix = 0;
-    st->bits = 0;
-    st->need = k;
-    st->done = (k == 0);
+__device__ void block_radix_select(const Get& get, int n, uint32_t k, SelectScratch& sc) {
+  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  uint64_t kmin = ~0ull, kmax = 0ull;
+  for (int i = tid; i < n; i += nt) {
+    const uint64_t key = get(i);
+    kmin = key < kmin ? key : kmin;
+    kmax = key > kmax ? key : kmax;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const uint64_t a = __shfl_xor_sync(0xFFFFFFFFu, kmin, off);
+    const uint64_t b = __shfl_xor_sync(0xFFFFFFFFu, kmax, off);
+    kmin = a < kmin ? a : kmin;
+    kmax = b > kmax ? b : kmax;
+  }
+  if (lane == 0) {
+    sc.red_min[warp] = kmin;
+    sc.red_max[warp] = kmax;
   }
   __syncthreads();
-  while (!st->done) {
-    const int bits = st->bits;
-    const uint64_t prefix = st->prefix;
-    const int shift = 56 - bits;
-    for (int i = tid; i < 256; i += nt) hist256[i] = 0;
+  if (tid == 0) {
+    for (int w = 1; w < (nt + 31) / 32; ++w) {
+      kmin = sc.red_min[w] < kmin ? sc.red_min[w] : kmin;
+      kmax = sc.red_max[w] > kmax ? sc.red_max[w] : kmax;
+    }
+    const int common = (kmin == kmax) ? 64 : __clzll(static_cast<long long>(kmin ^ kmax));
+    RadixState& st = sc.st;
+    st.bits = common;
+    st.prefix = common == 0 ? 0ull : (common == 64 ? kmax : (kmax & (~0ull << (64 - common))));
+    st.need = k;
+    st.done = (common == 64) || (static_cast<uint32_t>(n) == k);
+    if (static_cast<uint32_t>(n) == k) {  // everything is selected
+      st.bits = 0;
+      st.prefix = 0ull;
+    }
+  }
+  __syncthreads();
+  while (!sc.st.done) {
+    const int bits = sc.st.bits;
+    const uint64_t prefix = sc.st.prefix;
+    const int width = min(kDigitBits, 64 - bits);
+    const int shift = 64 - bits - width;
+    const uint64_t dmask = (1ull << width) - 1ull;
+    for (int i = tid; i < kDigitBins; i += nt) sc.hist[i] = 0;
     __syncthreads();
     for (int i = tid; i < n; i += nt) {
       const uint64_t key = get(i);
       if (bits == 0 || (key >> (64 - bits)) == (prefix >> (64 - bits)))
-        atomicAdd(&hist256[(key >> shift) & 255u], 1u);
+        atomicAdd(&sc.hist[static_cast<uint32_t>((key >> shift) & dmask)], 1u);
     }
     __syncthreads();
-    if (tid < 32) {
-      uint32_t above;
-      const int d = warp_find_digit256(hist256, st->need, &above);
-      if (tid == 0) {
-        const uint32_t need = st->need - above;
-        st->need = need;
-        st->prefix = prefix | (static_cast<uint64_t>(d) << shift);
-        st->bits = bits + 8;
-        st->done = (hist256[d] == need) || (bits + 8 == 64);
-      }
+    const uint32_t need = sc.st.need;
+    const int d = block_find_bin4096(sc.hist, need, sc.part, sc.ints);
+    if (tid == 0) {
+      const uint32_t left = need - static_cast<uint32_t>(sc.ints[3]);
+      sc.st.need = left;
+      sc.st.prefix = prefix | (static_cast<uint64_t>(d) << shift);
+      sc.st.bits = bits + width;
+      sc.st.done = (sc.hist[d] == left) || (bits + width == 64);
     }
     __syncthreads();
   }
@@ -148,6 +210,34 @@ __device__ void block_radix_select(const Get& get, int n, uint32_t k, uint32_t* 
 __device__ __forceinline__ bool radix_selected(uint64_t key, const RadixState& st) {
   if (st.bits == 0) return true;
   return (key >> (64 - st.bits)) >= (st.prefix >> (64 - st.bits));
+}
+
+// Order-preserving compaction over items 0..n-1 (whole CTA): emit(i, slot) is called for every
+// item with pred(i), slot counting those items in item order. Warp w owns a contiguous segment of
+// items and its lanes take consecutive items (conflict-free shared-memory reads); ballot prefix
+// counts keep the order inside a warp and a scan over the warps' totals orders the segments.
+// Returns the number of items emitted.
+template <class Pred, class Emit>
+__device__ uint32_t block_ordered_compact(int n, const Pred& pred, const Emit& emit,
+                                          uint32_t* scan_scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  const int seg = ((n + nw - 1) / nw + 31) & ~31;
+  const int lo = min(n, warp * seg), hi = min(n, lo + seg);
+  uint32_t c = 0;
+  for (int i = lo + lane; i < hi; i += 32) c += pred(i) ? 1u : 0u;
+  c = __reduce_add_sync(0xFFFFFFFFu, c);
+  uint32_t total;
+  // one value per thread: lane 0 carries the warp's count
+  const uint32_t warp_off = block_exclusive_scan(lane == 0 ? c : 0u, scan_scratch, &total);
+  uint32_t base = __shfl_sync(0xFFFFFFFFu, warp_off, 0);
+  for (int i0 = lo; i0 < hi; i0 += 32) {
+    const int i = i0 + lane;
+    const bool p = i < hi && pred(i);
+    const uint32_t ball = __ballot_sync(0xFFFFFFFFu, p);
+    if (p) emit(i, base + __popc(ball & ((1u << lane) - 1u)));
+    base += __popc(ball);
+  }
+  return total;
 }
 
 // Ascending bitonic sort of a[0..n2) in shared memory, n2 a power of two (whole CTA).

@@ -93,7 +93,7 @@ def make_case(B, n_cap, seed, kind="gauss"):
 @pytest.mark.parametrize("B,n_cap,N,K,P,kind", [
     (1, 4096, [4096], 64, 64, "gauss"),                      # the tiny Full-layer workload
     (3, 8320, [8320, 37, 5001], 512, 128, "gauss"),          # ragged N: partial tiles, N < K
-    (2, 20480, [20480, 19999], 512, 2048, "cluster"),        # P*8 < N < P*8... pool of all blocks
+    (2, 20480, [20480, 19999], 512, 2048, "cluster"),        # top 2048 of 2560 blocks
     (2, 16384, [16384, 12000], 256, 256, "ties"),            # many exact ties
 ])
 def test_full_index_matches_oracle(gpu, B, n_cap, N, K, P, kind):
@@ -104,8 +104,8 @@ def test_full_index_matches_oracle(gpu, B, n_cap, N, K, P, kind):
 
 
 def test_full_index_all_equal_scores_takes_lowest_indices(gpu):
-    """A zero query makes every score 0: ties go to the lowest positions. With N above the
-    candidate capacity this also exercises the exact select over the whole score array."""
+    """A zero query makes every score 0: ties go to the lowest positions and blocks, and every
+    block is a candidate of the select."""
     B, n_cap, K, P = 2, 40960, 512, 2048
     iq = torch.zeros(B, 4, 64, dtype=torch.bfloat16)
     w = torch.ones(B, 4)
@@ -117,6 +117,30 @@ def test_full_index_all_equal_scores_takes_lowest_indices(gpu):
         assert list(topk[b]) == list(range(K))
         assert list(pool[b]) == list(range(8 * P))
         assert np.all(scores[b, :N[b]] == 0) and not np.signbit(scores[b, :N[b]]).any()
+
+
+def test_full_index_candidates_beyond_shared_memory(gpu):
+    """Equal block maxima over 32,768 blocks: every block is a candidate (more than one CTA's
+    shared memory holds), so the select reads the chunked candidate regions from global memory."""
+    B, n_cap, K, P = 1, 262144, 64, 32
+    iq = torch.zeros(B, 4, 64, dtype=torch.bfloat16)
+    w = torch.ones(B, 4)
+    ik = torch.randn(B, n_cap, 64).to(torch.bfloat16)
+    topk, pool, scores, err = run_full(iq, w, ik, [n_cap], K, P, gpu)
+    assert err == 0
+    assert list(topk[0]) == list(range(K))
+    assert list(pool[0]) == list(range(8 * P))
+
+
+@pytest.mark.parametrize("K,P", [(512, 16), (100, 7)])
+def test_full_index_pool_smaller_than_topk(gpu, K, P):
+    """P < K: the Top-K comes from the top-K blocks while the pool keeps only the top P."""
+    B, n_cap = 2, 8192
+    iq, w, ik = make_case(B, n_cap, seed=K + P)
+    N = [8192, 6001]
+    topk, pool, scores, err = run_full(iq, w, ik, N, K, P, gpu)
+    assert err == 0
+    check_full(iq, w, ik, N, K, P, topk, pool, scores)
 
 
 def test_full_index_empty_and_tiny_sequences(gpu):
