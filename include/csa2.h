@@ -139,6 +139,25 @@ CSA2_API int csa2_index_reindex(const void *iq, const float *w, const void *ik_c
                        void *ws, size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream);
 
 /*
+ * Allocation-free Reindex-mode indexer (no counterpart on the pages; an interface addition).
+ * Same arguments and results as csa2_index_reindex without the workspace: for callers that may
+ * not allocate device memory where they run the decode step (a serving runtime that owns all
+ * device memory through its own pool, a plugin handed only its tensors, a latency-critical loop
+ * that cannot afford cudaMalloc's device-wide synchronisation). The scratch is a fixed array of
+ * CSA2_NOALLOC_REINDEX_MAX_SLOTS 8-byte slots (2 MiB) inside the library's device image, held by
+ * every GPU that loads the library until the process exits; B * L above that limit returns
+ * CSA2_ERR_UNSUPPORTED. The first call on a device looks up the array's device address for that
+ * device (make that first call before any stream capture). All calls on a device share the
+ * array: calls whose kernels overlap on the GPU race and must be serialised by the caller. The
+ * array needs no clearing: each call writes every slot it reads. It allocates nothing.
+ */
+enum { CSA2_NOALLOC_REINDEX_MAX_SLOTS = 262144 };
+CSA2_API int csa2_index_reindex_noalloc(const void *iq, const float *w, const void *ik_cache,
+                                        const int32_t *N, int B, int n_cap, const int32_t *pool,
+                                        int L, int K, int32_t *topk, int32_t *dev_err,
+                                        csa2_stream_t stream);
+
+/*
  * Sparse attention over the selected MXFP4 entries and the FP8 SWA rows, all 16 heads.
  * Defines: Reuse mode of section 一 ("sparse attention directly" over reused indices) and the
  * FP8 SWA KV. `mode` records which kind of layer produced idx; it does not change the result

@@ -49,6 +49,7 @@ def lib() -> ctypes.CDLL:
         L.csa2_index_reindex_workspace_bytes.argtypes = [I, I, I]
         L.csa2_index_reindex_workspace_bytes.restype = Z
         L.csa2_index_reindex.argtypes = [P, P, P, P, I, I, P, I, I, P, P, Z, P, P]
+        L.csa2_index_reindex_noalloc.argtypes = [P, P, P, P, I, I, P, I, I, P, P, P]
         L.csa2_attend_workspace_bytes.argtypes = [I, I, I]
         L.csa2_attend_workspace_bytes.restype = Z
         L.csa2_attend.argtypes = [I, P, ctypes.c_float, P, P, I, P, P, I, P, P, P, I, I, P, P, P,
@@ -144,6 +145,20 @@ def index_reindex(iq, w, ik_cache, N, pool, K, topk, ws, dev_err=None, stream=No
         _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _ptr(dev_err, torch.int32, "dev_err"),
         _stream(stream))
     _check("csa2_index_reindex", st)
+
+
+def index_reindex_noalloc(iq, w, ik_cache, N, pool, K, topk, dev_err=None, stream=None) -> None:
+    """Reindex-mode indexer without a workspace: the library uses its own fixed 2 MiB device
+    array (B * L up to 262,144 slots). For callers that cannot allocate device memory; calls that
+    overlap on one GPU share that array and must not run concurrently."""
+    B, n_cap = ik_cache.shape[0], ik_cache.shape[1]
+    L = pool.shape[1]
+    st = lib().csa2_index_reindex_noalloc(
+        _ptr(iq, torch.bfloat16, "iq"), _ptr(w, torch.float32, "w"),
+        _ptr(ik_cache, torch.bfloat16, "ik_cache"), _ptr(N, torch.int32, "N"), B, n_cap,
+        _ptr(pool, torch.int32, "pool"), L, K, _ptr(topk, torch.int32, "topk"),
+        _ptr(dev_err, torch.int32, "dev_err"), _stream(stream))
+    _check("csa2_index_reindex_noalloc", st)
 
 
 def attend_workspace_bytes(B: int, K: int, W: int) -> int:
