@@ -101,6 +101,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
 
+  // the first tile's indices load before the query prologue so the two latencies overlap
+  int pos_first[4] = {-1, -1, -1, -1};
+  if (t_begin < t_end && t_begin < tiles_idx) {
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+      const int item = pass * 16 + (tid >> 4);
+      if (item < min(kTile, K - t_begin * kTile))
+        pos_first[pass] = __ldg(idx + static_cast<int64_t>(b) * K + t_begin * kTile + item);
+    }
+  }
+
   // ---- q -> fp16 with a per-head power-of-two scale (16 threads per head, 32 dims each)
   {
     const int h = tid >> 4, r = tid & 15;
@@ -162,7 +173,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int pass = 0; pass < 4; ++pass) {
           const int item = pass * 16 + (tid >> 4);
-          pos[pass] = item < count ? __ldg(idx + static_cast<int64_t>(b) * K + base + item) : -1;
+          pos[pass] = tile == t_begin ? pos_first[pass]
+                      : (item < count ? __ldg(idx + static_cast<int64_t>(b) * K + base + item) : -1);
         }
         uint4 cw[4];
         uint32_t sw[4];
@@ -245,9 +257,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (lane == 0) sm.tile_pf = smax > 0.0f ? pow2f(-ilog2f(smax)) : 1.0f;
     }
 
-    // ---- logits: warp w computes z[0..16)[8w .. 8w+8)
+    // ---- logits: warp w computes z[0..16)[8w .. 8w+8); even and odd k-steps accumulate in two
+    // independent chains
     {
-      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc2[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       const int mi = lane >> 3;
       const int a_row = (lane & 7) + ((mi & 1) << 3);
       const int v_row = 8 * warp + (lane & 7);
@@ -258,8 +271,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         ldsm_x4(q_base + swz1024(a_row, 2 * s + 2 + (mi >> 1)), a4, a5, a6, a7);
         ldsm_x4(v_base + swz1024(v_row, 2 * s + mi), b0, b1, b2, b3);
         mma_f16_16816(acc, a0, a1, a2, a3, b0, b1);
-        mma_f16_16816(acc, a4, a5, a6, a7, b2, b3);
+        mma_f16_16816(acc2, a4, a5, a6, a7, b2, b3);
       }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] += acc2[k];
       const int i0 = 8 * warp + 2 * c, i1 = i0 + 1;
       const float u0 = sm.q_unscale[g], u1 = sm.q_unscale[g + 8];
       const float s0 = sm.item_scale[i0], s1 = sm.item_scale[i1];

@@ -20,11 +20,12 @@
 //                       per 8192-block chunk.
 //   index_final_kernel  one CTA per sequence: radix select of the top max(K, P) blocks over the
 //                       candidates, order-preserving compaction (ascending block ids, no sort),
-//                       the pool (top P blocks), then the position Top-K over the scores of the
-//                       selected blocks' positions. Every Top-K position lies in one of the top
-//                       max(K, P) blocks: a block ranked above the block of a selected position
-//                       holds its own maximum, which outranks that position, so fewer than K
-//                       blocks outrank it.
+//                       the pool (top P blocks), then the position Top-K over the positions of
+//                       those blocks: the score gather histograms 12 key bits and only positions
+//                       at or above the K-th score's bin enter the radix select. Every Top-K
+//                       position lies in one of the top max(K, P) blocks: a block ranked above
+//                       the block of a selected position holds its own maximum, which outranks
+//                       that position, so fewer than K blocks outrank it.
 // Every mbarrier wait is bounded; a timeout flags CSA2_DEVERR_TIMEOUT and the CTA drains its own
 // bulk copies before exiting.
 #include <mutex>
@@ -282,7 +283,7 @@ __global__ void __launch_bounds__(kCollectThreads)
   constexpr int kPer = kCollectChunk / kCollectThreads;  // 32 blocks per thread
   __shared__ uint32_t part[kCollectThreads];
   __shared__ uint32_t scan[33];
-  __shared__ int sh[4];
+  __shared__ int sh[6];
   pdl_wait();
   pdl_launch_dependents();
   const int b = blockIdx.y, chunk = blockIdx.x;
@@ -333,12 +334,10 @@ struct FinalSmem {
     uint32_t skey[2 * kSmemKeys];    // score keys of the selected blocks' positions
   } u;
   int32_t wide[kMaxSel];             // top max(K, P) blocks, ascending
-  uint64_t wide_key[kMaxSel];        // their rank keys
+  uint64_t wide_key[kMaxSel];        // their rank keys; later the position candidates
   union {
     int32_t chunk_pre[kMaxSel + 1];  // candidate prefix over chunks (while loading candidates)
-    int32_t pos_blk[kMaxSel];        // top-K blocks (hold every Top-K position), ascending
   } v;
-  uint8_t flag[kMaxSel];             // bit 0: wide[i] is in the pool; bit 1: in the top-K blocks
   SelectScratch sc;
 };
 
@@ -457,26 +456,14 @@ __global__ void __launch_bounds__(kFinalThreads)
         },
         sm.sc.scan);
   }
-  for (int i = tid; i < kw; i += kFinalThreads) sm.flag[i] = 3;
-  __syncthreads();
-
-  // ---- the pool (top kp blocks) and the position blocks (top kkb blocks) are the top parts of
-  // the wide set; the smaller of the two is selected again among the wide keys
-  const int kkb = min(K, nbl);
+  // ---- the pool: the top kp blocks, i.e. the whole wide set unless P < K
   const uint64_t* wk = sm.wide_key;
-  auto wide_key = [wk](int i) { return wk[i]; };
-  if (kp < kw || kkb < kw) {
-    const int ksub = kp < kw ? kp : kkb;
-    const uint8_t clear = kp < kw ? 1 : 2;
-    block_radix_select(wide_key, kw, static_cast<uint32_t>(ksub), sm.sc);
+  if (kp < kw) {
+    auto wide_key = [wk](int i) { return wk[i]; };
+    block_radix_select(wide_key, kw, static_cast<uint32_t>(kp), sm.sc);
     const RadixState st = sm.sc.st;
-    for (int i = tid; i < kw; i += kFinalThreads)
-      if (!radix_selected(wk[i], st)) sm.flag[i] &= static_cast<uint8_t>(~clear);
-    __syncthreads();
-  }
-  {
     const uint32_t n_pool = block_ordered_compact(
-        kw, [&](int i) { return (sm.flag[i] & 1) != 0; },
+        kw, [&](int i) { return radix_selected(wk[i], st); },
         [&](int i, uint32_t slot) {
           for (int r = 0; r < S; ++r) {
             const int p = sm.wide[i] * S + r;
@@ -486,127 +473,158 @@ __global__ void __launch_bounds__(kFinalThreads)
         sm.sc.scan);
     for (int i = static_cast<int>(n_pool) * S + tid; i < P * S; i += kFinalThreads)
       pool_out[i] = -1;
-    block_ordered_compact(
-        kw, [&](int i) { return (sm.flag[i] & 2) != 0; },
-        [&](int i, uint32_t slot) { sm.v.pos_blk[slot] = sm.wide[i]; }, sm.sc.scan);
+  } else {
+    for (int i = tid; i < P * S; i += kFinalThreads) {
+      const int j = i / S;
+      const int p = j < kw ? sm.wide[j] * S + (i % S) : nb;
+      pool_out[i] = p < nb ? p : -1;
+    }
   }
-  __syncthreads();
 
-  // ---- position Top-K over the top-K blocks' positions (slot order = ascending position)
-  const int L = kkb * S;
+  // ---- position Top-K over every position of the wide blocks (slot order = ascending
+  // position). The score gather also histograms the top 12 bits of each score key; only the
+  // positions at or above the bin that holds the K-th score enter the radix select.
+  const int L = kw * S;  // <= 32768
   const float* srow = scores + static_cast<int64_t>(b) * n_cap;
-  const bool keys64 = L <= kSmemKeys;
+  for (int i = tid; i < kDigitBins; i += kFinalThreads) sm.sc.hist[i] = 0u;
+  __syncthreads();
   for (int base = 0; base < L; base += 8 * kFinalThreads) {
     float vals[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int i = base + j * kFinalThreads + tid;
-      const int p = i < L ? sm.v.pos_blk[i / S] * S + (i % S) : nb;
+      const int p = i < L ? sm.wide[i / S] * S + (i % S) : nb;
       vals[j] = p < nb ? __ldg(srow + p) : 0.0f;
     }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int i = base + j * kFinalThreads + tid;
       if (i < L) {
-        const uint32_t p = static_cast<uint32_t>(sm.v.pos_blk[i / S] * S + (i % S));
-        const bool valid = p < static_cast<uint32_t>(nb);
-        if (keys64) sm.u.cand[i] = valid ? rank_key(vals[j], p) : 0ull;
-        else sm.u.skey[i] = valid ? float_key(vals[j]) : 0u;
+        const int p = sm.wide[i / S] * S + (i % S);
+        const uint32_t key = p < nb ? float_key(vals[j]) : 0u;  // 0: below every real key
+        sm.u.skey[i] = key;
+        if (p < nb) atomicAdd(&sm.sc.hist[key >> kHistShift], 1u);
       }
     }
   }
   __syncthreads();
+  auto pos_of = [&](int i) { return static_cast<uint32_t>(sm.wide[i / S] * S + (i % S)); };
   auto pos_key = [&](int i) -> uint64_t {
-    if (keys64) return sm.u.cand[i];
     const uint32_t hk = sm.u.skey[i];
-    if (hk == 0u) return 0ull;  // a position past N: below every real key
-    const uint32_t p = static_cast<uint32_t>(sm.v.pos_blk[i / S] * S + (i % S));
-    return (static_cast<uint64_t>(hk) << 32) | static_cast<uint64_t>(~p);
+    return hk == 0u ? 0ull : (static_cast<uint64_t>(hk) << 32) | static_cast<uint64_t>(~pos_of(i));
   };
-  block_radix_select(pos_key, L, static_cast<uint32_t>(kk), sm.sc);
-  {
+  const int T0 = block_find_bin4096(sm.sc.hist, static_cast<uint32_t>(kk), sm.sc.part, sm.sc.ints);
+  // candidates in slot order into the (now free) wide_key array
+  uint64_t* cbuf = sm.wide_key;
+  const uint32_t n_cand = block_ordered_compact(
+      L, [&](int i) { const uint32_t k = sm.u.skey[i]; return k != 0u && static_cast<int>(k >> kHistShift) >= T0; },
+      [&](int i, uint32_t slot) { if (slot < kMaxSel) cbuf[slot] = pos_key(i); }, sm.sc.scan);
+  __syncthreads();
+  uint32_t n_sel;
+  if (n_cand <= static_cast<uint32_t>(kMaxSel)) {
+    auto get = [cbuf](int i) { return cbuf[i]; };
+    block_radix_select(get, static_cast<int>(n_cand), static_cast<uint32_t>(kk), sm.sc);
     const RadixState st = sm.sc.st;
-    const uint32_t n_sel = block_ordered_compact(
-        L, [&](int i) { const uint64_t k = pos_key(i); return k != 0ull && radix_selected(k, st); },
+    n_sel = block_ordered_compact(
+        static_cast<int>(n_cand), [&](int i) { return radix_selected(cbuf[i], st); },
         [&](int i, uint32_t slot) {
-          if (slot < static_cast<uint32_t>(K)) topk_out[slot] = sm.v.pos_blk[i / S] * S + (i % S);
+          if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(rank_key_index(cbuf[i]));
         },
         sm.sc.scan);
-    for (int i = static_cast<int>(n_sel) + tid; i < K; i += kFinalThreads) topk_out[i] = -1;
+  } else {
+    block_radix_select(pos_key, L, static_cast<uint32_t>(kk), sm.sc);
+    const RadixState st = sm.sc.st;
+    n_sel = block_ordered_compact(
+        L, [&](int i) { const uint64_t k = pos_key(i); return k != 0ull && radix_selected(k, st); },
+        [&](int i, uint32_t slot) {
+          if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(pos_of(i));
+        },
+        sm.sc.scan);
   }
+  for (int i = static_cast<int>(n_sel) + tid; i < K; i += kFinalThreads) topk_out[i] = -1;
 }
 
 // ------------------------------------------------------------------------------------ Reindex
 
-constexpr int kReSlotsPerCta = 256;
-constexpr int kReThreads = 256;
+// Reindex scoring on the tensor cores. A warp takes tiles of 16 pool slots: lane (g, c) loads 32
+// contiguous bytes (dims 16c .. 16c+15) of the keys of slots g and g+8 straight into registers,
+// which is the m16n8k16 A fragment under a permutation of the 64 dims (k-step s, pair 2c ->
+// dims 16c+4s, +1; pair 2c+8 -> dims 16c+4s+2, +3); the query fragments use the same permutation.
+// All pool entries, then all key rows of a warp's tiles are loaded before any arithmetic.
+constexpr int kReWarps = 8;
+constexpr int kReThreads = kReWarps * 32;
+constexpr int kReTilesPerWarp = 4;
+constexpr int kReSlotsPerCta = kReWarps * kReTilesPerWarp * 16;  // 512
 
-// 8 lanes per pool slot, 8 dims (16 bytes of key) per lane; writes the slot's rank key (0 for an
-// empty or out-of-range slot, which is below every real key).
-__global__ void __launch_bounds__(kReThreads, 3)
+__global__ void __launch_bounds__(kReThreads)
     reindex_score_kernel(const uint16_t* __restrict__ iq, const float* __restrict__ w,
                          const uint16_t* __restrict__ ik_cache, const int32_t* __restrict__ N,
                          int n_cap, const int32_t* __restrict__ pool, int L,
                          uint64_t* __restrict__ keys, int32_t* dev_err) {
-  __shared__ float qs[HI][DI];
-  __shared__ float wh[HI];
   pdl_wait();
   pdl_launch_dependents();
   const int b = blockIdx.y;
-  const int lane = threadIdx.x & 31, sub = lane & 7;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, c = lane & 3;
   const int nb = clamp_len(N, b, n_cap, threadIdx.x == 0 && blockIdx.x == 0 ? dev_err : nullptr);
+  // query fragments: head g (< 4) of iq[b] under the dim permutation; heads 4..7 are zero
+  uint32_t bq0[4], bq1[4];
   {
-    const int h = threadIdx.x >> 6, i = threadIdx.x & 63;  // 256 threads = 4 heads x 64 dims
-    const uint16_t qb = iq[(static_cast<int64_t>(b) * HI + h) * DI + i];
-    qs[h][i] = __uint_as_float(static_cast<uint32_t>(qb) << 16);
-    if (threadIdx.x < HI) wh[threadIdx.x] = __ldg(w + b * HI + threadIdx.x);
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(iq + (static_cast<int64_t>(b) * HI + min(g, HI - 1)) * DI);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      bq0[s] = g < HI ? __ldg(qrow + 8 * c + 2 * s) : 0u;
+      bq1[s] = g < HI ? __ldg(qrow + 8 * c + 2 * s + 1) : 0u;
+    }
   }
-  __syncthreads();
-  const int slot0 = blockIdx.x * kReSlotsPerCta;
-  const int slot_end = min(slot0 + kReSlotsPerCta, L);
-  constexpr int per_iter = kReThreads / 8;
-  constexpr int kIter = kReSlotsPerCta / per_iter;
-  // all pool loads, then all key loads, then the arithmetic (two memory round trips per CTA)
-  int pos[kIter];
+  const float wa = c < 2 ? __ldg(w + b * HI + 2 * c) : 0.0f;
+  const float wb = c < 2 ? __ldg(w + b * HI + 2 * c + 1) : 0.0f;
+  const int slot0 = blockIdx.x * kReSlotsPerCta + warp * kReTilesPerWarp * 16;
+  const int32_t* prow = pool + static_cast<int64_t>(b) * L;
+  int pos[kReTilesPerWarp][2];
 #pragma unroll
-  for (int it = 0; it < kIter; ++it) {
-    const int s = slot0 + it * per_iter + (threadIdx.x >> 3);
-    pos[it] = s < slot_end ? __ldg(pool + static_cast<int64_t>(b) * L + s) : -1;
-  }
-  uint4 u[kIter];
+  for (int t = 0; t < kReTilesPerWarp; ++t)
 #pragma unroll
-  for (int it = 0; it < kIter; ++it) {
-    const bool valid = pos[it] >= 0 && pos[it] < nb;
-    if (!valid && pos[it] != -1 && sub == 0) flag_error(dev_err, CSA2_DEVERR_INDEX_RANGE);
-    u[it] = valid ? ldg_nc_v4(reinterpret_cast<const uint4*>(
-                        ik_cache + (static_cast<int64_t>(b) * n_cap + pos[it]) * DI) + sub)
-                  : make_uint4(0u, 0u, 0u, 0u);
-  }
+    for (int h = 0; h < 2; ++h) {
+      const int s = slot0 + 16 * t + g + 8 * h;
+      pos[t][h] = s < L ? __ldg(prow + s) : -1;
+    }
+  uint4 u[kReTilesPerWarp][2][2];
 #pragma unroll
-  for (int it = 0; it < kIter; ++it) {
-    const int s = slot0 + it * per_iter + (threadIdx.x >> 3);
-    const bool valid = pos[it] >= 0 && pos[it] < nb;
-    const uint32_t uw[4] = {u[it].x, u[it].y, u[it].z, u[it].w};
-    float d[HI] = {0.0f, 0.0f, 0.0f, 0.0f};
+  for (int t = 0; t < kReTilesPerWarp; ++t)
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float x0 = bf16lo(uw[k]), x1 = bf16hi(uw[k]);
-#pragma unroll
-      for (int h = 0; h < HI; ++h)
-        d[h] = fmaf(qs[h][8 * sub + 2 * k + 1], x1, fmaf(qs[h][8 * sub + 2 * k], x0, d[h]));
+    for (int h = 0; h < 2; ++h) {
+      const int p = pos[t][h];
+      const bool valid = p >= 0 && p < nb;
+      if (!valid && p != -1 && c == 0) flag_error(dev_err, CSA2_DEVERR_INDEX_RANGE);
+      const uint4* src = reinterpret_cast<const uint4*>(
+                             ik_cache + (static_cast<int64_t>(b) * n_cap + (valid ? p : 0)) * DI) + 2 * c;
+      u[t][h][0] = valid ? ldg_nc_v4(src) : make_uint4(0u, 0u, 0u, 0u);
+      u[t][h][1] = valid ? ldg_nc_v4(src + 1) : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int h = 0; h < HI; ++h) {
-      d[h] += __shfl_xor_sync(0xFFFFFFFFu, d[h], 1);
-      d[h] += __shfl_xor_sync(0xFFFFFFFFu, d[h], 2);
-      d[h] += __shfl_xor_sync(0xFFFFFFFFu, d[h], 4);
-    }
-    if (sub == 0 && s < slot_end) {
-      float score = 0.0f;
+  for (int t = 0; t < kReTilesPerWarp; ++t) {
+    const uint32_t r0[8] = {u[t][0][0].x, u[t][0][0].y, u[t][0][0].z, u[t][0][0].w,
+                            u[t][0][1].x, u[t][0][1].y, u[t][0][1].z, u[t][0][1].w};
+    const uint32_t r1[8] = {u[t][1][0].x, u[t][1][0].y, u[t][1][0].z, u[t][1][0].w,
+                            u[t][1][1].x, u[t][1][1].y, u[t][1][1].z, u[t][1][1].w};
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int h = 0; h < HI; ++h) score = fmaf(wh[h], fmaxf(d[h], 0.0f), score);
-      keys[static_cast<int64_t>(b) * L + s] =
-          valid ? rank_key(score, static_cast<uint32_t>(pos[it])) : 0ull;
+    for (int s = 0; s < 4; ++s)
+      mma_bf16_16816(acc, r0[2 * s], r1[2 * s], r0[2 * s + 1], r1[2 * s + 1], bq0[s], bq1[s]);
+    float s0 = wa * fmaxf(acc[0], 0.0f) + wb * fmaxf(acc[1], 0.0f);
+    float s1 = wa * fmaxf(acc[2], 0.0f) + wb * fmaxf(acc[3], 0.0f);
+    s0 += __shfl_xor_sync(0xFFFFFFFFu, s0, 1);
+    s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
+    if (c == 0) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int s = slot0 + 16 * t + g + 8 * h;
+        const int p = pos[t][h];
+        if (s < L)
+          keys[static_cast<int64_t>(b) * L + s] =
+              (p >= 0 && p < nb) ? rank_key(h ? s1 : s0, static_cast<uint32_t>(p)) : 0ull;
+      }
     }
   }
 }
@@ -851,7 +869,7 @@ cudaError_t launch_index_reindex(const void* iq, const float* w, const void* ik_
     cudaError_t e = set_smem(reindex_final_kernel, sizeof(ReFinalSmem), done);
     if (e != cudaSuccess) return e;
   }
-  const dim3 grid((L + kReSlotsPerCta - 1) / kReSlotsPerCta, B);
+  const dim3 grid((L + kReSlotsPerCta - 1) / kReSlotsPerCta, B);  // 32 CTAs per 16,384 slots
   profile_begin(CSA2_KERNEL_REINDEX, s);
   cudaError_t e = launch_pdl(reindex_score_kernel, grid, dim3(kReThreads), 0, s,
                              static_cast<const uint16_t*>(iq), w,

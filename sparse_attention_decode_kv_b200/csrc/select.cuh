@@ -55,70 +55,70 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
 // ------------------------------------------------------------------------------ threshold bin
 
 // The largest bin T of a 4096-bin histogram with sum_{bins >= T} >= need (whole CTA; blockDim.x
-// divides 4096 and is at least 256). `hist` may live in global or shared memory. Every thread
-// loads its contiguous bins at once; the owners of the crossing group resolve the exact bin.
+// is 256 or 1024, so each thread owns 16 or 4 consecutive bins). `hist` may live in global or
+// shared memory. Three parallel levels: warp sums, then the crossing warp's thread sums, then the
+// crossing thread's bins (kept in registers). part: >= 32 shared words; shared_int: 6 words;
 // shared_int[3] receives the count in the bins above T.
 __device__ __forceinline__ int block_find_bin4096(const uint32_t* hist, uint32_t need,
                                                   uint32_t* part, int* shared_int) {
-  const int tid = threadIdx.x, nt = blockDim.x;
-  const int per = kHistBins / nt;  // 4 (1024 threads) or 16 (256 threads)
+  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = nt >> 5;
+  const int per = kHistBins / nt;
   uint32_t h[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) h[i] = i < per ? hist[tid * per + i] : 0u;
   uint32_t s = 0;
 #pragma unroll
   for (int i = 0; i < 16; ++i) s += h[i];
-  part[tid] = s;
+  const uint32_t wsum = __reduce_add_sync(0xFFFFFFFFu, s);
+  if (lane == 0) part[warp] = wsum;
   __syncthreads();
-  if (tid < 32) {
-    const int pl = nt / 32;  // parts per lane
-    uint32_t q = 0;
-    for (int i = 0; i < pl; ++i) q += part[tid * pl + i];
-    uint32_t suf = q;
+  if (warp == 0) {
+    const uint32_t v = lane < nw ? part[lane] : 0u;
+    uint32_t suf = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, suf, off);
-      if (tid + off < 32) suf += v;
+      const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, suf, off);
+      if (lane + off < 32) suf += y;
     }
-    const uint32_t ball = __ballot_sync(0xFFFFFFFFu, suf >= need);
-    const int L = ball ? 31 - __clz(ball) : 0;
-    uint32_t run = __shfl_sync(0xFFFFFFFFu, suf, (L + 1) & 31);
-    if (L == 31) run = 0;
-    // lane L's parts, resolved by the whole warp (at most 32 parts per lane)
-    const uint32_t pv = tid < pl ? part[L * pl + tid] : 0u;
-    uint32_t psuf = pv;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, psuf, off);
-      if (tid + off < 32) psuf += v;
-    }
-    const uint32_t pball = __ballot_sync(0xFFFFFFFFu, tid < pl && run + psuf >= need);
-    const int j = pball ? 31 - __clz(pball) : 0;
-    const uint32_t above = __shfl_sync(0xFFFFFFFFu, psuf - pv, j);
-    if (tid == 0) {
-      shared_int[0] = L * pl + j;
-      shared_int[1] = static_cast<int>(run + above);  // count in the parts above that part
+    const uint32_t ball = __ballot_sync(0xFFFFFFFFu, lane < nw && suf >= need);
+    const int wl = ball ? 31 - __clz(ball) : 0;
+    const uint32_t above = __shfl_sync(0xFFFFFFFFu, suf - v, wl);
+    if (lane == 0) {
+      shared_int[0] = wl;
+      shared_int[1] = static_cast<int>(above);
     }
   }
   __syncthreads();
-  if (tid == shared_int[0]) {
-    uint32_t run = static_cast<uint32_t>(shared_int[1]);
-    int bin = tid * per;
+  if (warp == shared_int[0]) {
+    const uint32_t run = static_cast<uint32_t>(shared_int[1]);
+    uint32_t suf = s;
 #pragma unroll
-    for (int i = 15; i >= 0; --i) {
-      if (i >= per) continue;
-      if (run + h[i] >= need) {
-        bin = tid * per + i;
-        break;
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, suf, off);
+      if (lane + off < 32) suf += y;
+    }
+    const uint32_t ball = __ballot_sync(0xFFFFFFFFu, run + suf >= need);
+    const int jl = ball ? 31 - __clz(ball) : 0;
+    const uint32_t above = __shfl_sync(0xFFFFFFFFu, suf - s, jl);
+    if (lane == jl) {
+      uint32_t r = run + above;
+      int bin = tid * per;
+#pragma unroll
+      for (int i = 15; i >= 0; --i) {
+        if (i >= per) continue;
+        if (r + h[i] >= need) {
+          bin = tid * per + i;
+          break;
+        }
+        r += h[i];
       }
-      run += h[i];
+      shared_int[2] = bin;
+      shared_int[3] = static_cast<int>(r);
     }
-    shared_int[2] = bin;
-    shared_int[3] = static_cast<int>(run);
   }
   __syncthreads();
-  const int r = shared_int[2];
-  return r;
+  return shared_int[2];
 }
 
 // ------------------------------------------------------------------------------ radix select
@@ -134,7 +134,7 @@ struct SelectScratch {
   uint32_t hist[kDigitBins];
   uint32_t part[1024];
   uint32_t scan[33];
-  int ints[4];
+  int ints[6];
   uint64_t red_min[32], red_max[32];
   RadixState st;
 };
@@ -163,11 +163,19 @@ __device__ void block_radix_select(const Get& get, int n, uint32_t k, SelectScra
     sc.red_max[warp] = kmax;
   }
   __syncthreads();
-  if (tid == 0) {
-    for (int w = 1; w < (nt + 31) / 32; ++w) {
-      kmin = sc.red_min[w] < kmin ? sc.red_min[w] : kmin;
-      kmax = sc.red_max[w] > kmax ? sc.red_max[w] : kmax;
+  if (warp == 0) {
+    const int nw = (nt + 31) / 32;
+    kmin = lane < nw ? sc.red_min[lane] : ~0ull;
+    kmax = lane < nw ? sc.red_max[lane] : 0ull;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const uint64_t a = __shfl_xor_sync(0xFFFFFFFFu, kmin, off);
+      const uint64_t b = __shfl_xor_sync(0xFFFFFFFFu, kmax, off);
+      kmin = a < kmin ? a : kmin;
+      kmax = b > kmax ? b : kmax;
     }
+  }
+  if (tid == 0) {
     const int common = (kmin == kmax) ? 64 : __clzll(static_cast<long long>(kmin ^ kmax));
     RadixState& st = sc.st;
     st.bits = common;
@@ -216,7 +224,7 @@ __device__ __forceinline__ bool radix_selected(uint64_t key, const RadixState& s
 // item with pred(i), slot counting those items in item order. Warp w owns a contiguous segment of
 // items and its lanes take consecutive items (conflict-free shared-memory reads); ballot prefix
 // counts keep the order inside a warp and a scan over the warps' totals orders the segments.
-// Returns the number of items emitted.
+// Returns the number of items emitted; everything emitted is visible to the whole CTA on return.
 template <class Pred, class Emit>
 __device__ uint32_t block_ordered_compact(int n, const Pred& pred, const Emit& emit,
                                           uint32_t* scan_scratch) {
@@ -237,6 +245,7 @@ __device__ uint32_t block_ordered_compact(int n, const Pred& pred, const Emit& e
     if (p) emit(i, base + __popc(ball & ((1u << lane) - 1u)));
     base += __popc(ball);
   }
+  __syncthreads();
   return total;
 }
 
