@@ -66,6 +66,25 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def scan_traffic_per_launch(wl):
+    """DRAM bytes per scan launch from the committed ncu capture (profiles/index_scan_traffic.json),
+    scaled by entries scored; None once the scan kernel's source differs from the captured one."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "index_scan_traffic.json")) as f:
+            cap = json.load(f)
+        csrc = os.path.join(ROOT, "sparse_attention_decode_kv_b200", "csrc")
+        src = open(os.path.join(csrc, "index.cu")).read()
+        a = src.index("__global__ void __launch_bounds__(kScanThreads, 1)")
+        b = src.index("\n}\n", a) + 3
+        region = src[a:b] + open(os.path.join(csrc, "common.cuh")).read()
+        if hashlib.sha256(region.encode()).hexdigest() != cap["source_sha256"]:
+            return None
+        return int(round(cap["dram_bytes_per_entry"] * wl.B * wl.N))
+    except Exception:
+        return None
+
+
 def algorithmic_bytes(wl) -> dict:
     """Bytes the step must move (indexer keys + gathered MXFP4 entries + scales + SWA rows)."""
     full = wl.B * wl.N * 128
@@ -356,7 +375,8 @@ def run_ours(args, world, rank, local):
                      "achieved": round(scan_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(scan_gbs / peak, 4), "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": ab["full"],
-                     "launch_ms": round(scan_ms, 4), "traffic": None},
+                     "launch_ms": round(scan_ms, 4), "traffic": scan_traffic_per_launch(wl),
+                     "traffic_source": "profiles/index_scan_traffic.json (ncu, scaled by entries)"},
         "gpu_launches": per_step_launches * K,
         "clocks": clocks.summary(),
     }
