@@ -38,7 +38,7 @@ struct __align__(16) AttendSmem {
   uint16_t q[HQ * D];        // fp16 [16][512], 16-byte chunks XOR-swizzled by (row & 7)
   uint16_t v[kTile * D];     // fp16 [64][512], same swizzle
   uint16_t p[HQ * kTile];    // fp16 [16][64], same swizzle (8 chunks per row)
-  float z[HQ * kTile];       // logits of the current tile
+  float zp[2][HQ * kTile];   // partial logits of the current tile over dims 0..255 / 256..511
   float item_scale[kTile];   // 1 (MXFP4) or the SWA token's fp32 scale
   int item_valid[kTile];
   float q_unscale[HQ];       // 2^(e_h - 14) * softmax_scale
@@ -257,32 +257,34 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (lane == 0) sm.tile_pf = smax > 0.0f ? pow2f(-ilog2f(smax)) : 1.0f;
     }
 
-    // ---- logits: warp w computes z[0..16)[8w .. 8w+8); even and odd k-steps accumulate in two
-    // independent chains
+    // ---- logits: warp w takes items 16 (w % 4) .. +15 (two n-blocks, two independent
+    // accumulator chains) over dims 256 (w / 4) .. +255, so each warp reads half of q; the two
+    // halves are added in the softmax
     {
-      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc2[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      float acc0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, acc1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      const int ig = warp & 3, kh = warp >> 2;
       const int mi = lane >> 3;
       const int a_row = (lane & 7) + ((mi & 1) << 3);
-      const int v_row = 8 * warp + (lane & 7);
+      const int v_row = 16 * ig + (lane & 7) + ((lane >> 4) << 3);
+      const int v_sub = mi & 1;
 #pragma unroll 4
-      for (int s = 0; s < D / 16; s += 2) {
-        uint32_t a0, a1, a2, a3, a4, a5, a6, a7, b0, b1, b2, b3;
+      for (int s = 16 * kh; s < 16 * kh + 16; ++s) {
+        uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
         ldsm_x4(q_base + swz1024(a_row, 2 * s + (mi >> 1)), a0, a1, a2, a3);
-        ldsm_x4(q_base + swz1024(a_row, 2 * s + 2 + (mi >> 1)), a4, a5, a6, a7);
-        ldsm_x4(v_base + swz1024(v_row, 2 * s + mi), b0, b1, b2, b3);
-        mma_f16_16816(acc, a0, a1, a2, a3, b0, b1);
-        mma_f16_16816(acc2, a4, a5, a6, a7, b2, b3);
+        ldsm_x4(v_base + swz1024(v_row, 2 * s + v_sub), b0, b1, b2, b3);
+        mma_f16_16816(acc0, a0, a1, a2, a3, b0, b1);
+        mma_f16_16816(acc1, a0, a1, a2, a3, b2, b3);
       }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] += acc2[k];
-      const int i0 = 8 * warp + 2 * c, i1 = i0 + 1;
-      const float u0 = sm.q_unscale[g], u1 = sm.q_unscale[g + 8];
-      const float s0 = sm.item_scale[i0], s1 = sm.item_scale[i1];
-      const bool v0 = sm.item_valid[i0], v1 = sm.item_valid[i1];
-      sm.z[g * kTile + i0] = v0 ? acc[0] * u0 * s0 : -INFINITY;
-      sm.z[g * kTile + i1] = v1 ? acc[1] * u0 * s1 : -INFINITY;
-      sm.z[(g + 8) * kTile + i0] = v0 ? acc[2] * u1 * s0 : -INFINITY;
-      sm.z[(g + 8) * kTile + i1] = v1 ? acc[3] * u1 * s1 : -INFINITY;
+      float* zp = sm.zp[kh];
+      const int i0 = 16 * ig + 2 * c;
+      zp[g * kTile + i0] = acc0[0];
+      zp[g * kTile + i0 + 1] = acc0[1];
+      zp[(g + 8) * kTile + i0] = acc0[2];
+      zp[(g + 8) * kTile + i0 + 1] = acc0[3];
+      zp[g * kTile + i0 + 8] = acc1[0];
+      zp[g * kTile + i0 + 9] = acc1[1];
+      zp[(g + 8) * kTile + i0 + 8] = acc1[2];
+      zp[(g + 8) * kTile + i0 + 9] = acc1[3];
     }
     __syncthreads();
 
@@ -292,7 +294,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const int h = 2 * warp + hh;
-        const float z0 = sm.z[h * kTile + lane], z1 = sm.z[h * kTile + lane + 32];
+        const float uh = sm.q_unscale[h];
+        const float z0 = sm.item_valid[lane]
+                             ? (sm.zp[0][h * kTile + lane] + sm.zp[1][h * kTile + lane]) * uh * sm.item_scale[lane]
+                             : -INFINITY;
+        const float z1 = sm.item_valid[lane + 32]
+                             ? (sm.zp[0][h * kTile + lane + 32] + sm.zp[1][h * kTile + lane + 32]) * uh *
+                                   sm.item_scale[lane + 32]
+                             : -INFINITY;
         float mt = fmaxf(z0, z1);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, off));
@@ -392,58 +401,67 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-// Log-sum-exp merge of the split partials: grid = (16 heads, B), 128 threads x 4 dims. The
-// (m, l) pairs of all splits are read at once into shared memory, then every thread issues its
-// partial loads in groups of 8 independent requests.
+// Log-sum-exp merge of the split partials: grid = (16 heads, B), 128 threads x 4 dims. Every
+// thread requests the partial (m, l) it owns and its float4 of every split's partial o at once
+// (one memory round trip), then the weights exp(m_s - m) / l are formed in shared memory.
 constexpr int kMaxSplits = 128;
+constexpr int kMergeBatch = 16;  // partial-o requests in flight per thread
 __global__ void __launch_bounds__(128)
     attend_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                         int nsplit, float* __restrict__ out, float* __restrict__ lse) {
   __shared__ float wgt[kMaxSplits];
-  __shared__ float ml[2];
-  const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+  __shared__ float red[8];
+  const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   pdl_wait();
   pdl_launch_dependents();
   const int64_t p0 = static_cast<int64_t>(b) * nsplit;
   float ms = -INFINITY, ls = 0.0f;
   if (t < nsplit) {
-    ms = __ldg(part_ml + ((p0 + t) * HQ + h) * 2);
-    ls = __ldg(part_ml + ((p0 + t) * HQ + h) * 2 + 1);
+    const float2 ml = __ldg(reinterpret_cast<const float2*>(part_ml) + (p0 + t) * HQ + h);
+    ms = ml.x;
+    ls = ml.y;
   }
+  const float4* src = reinterpret_cast<const float4*>(part_o + (p0 * HQ + h) * D) + t;
+  const int64_t stride = static_cast<int64_t>(HQ) * D / 4;  // float4 between splits
+  float4 v[kMergeBatch];
+#pragma unroll
+  for (int j = 0; j < kMergeBatch; ++j)
+    v[j] = j < nsplit ? __ldg(src + j * stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+  // m = max over splits, l = sum exp(m_s - m) l_s (nsplit <= 128 = blockDim)
   float m = ms;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
-  if ((t & 31) == 0) wgt[t >> 5] = m;  // per-warp max (nsplit <= 128 = blockDim)
+  if (lane == 0) red[warp] = m;
   __syncthreads();
-  m = fmaxf(fmaxf(wgt[0], wgt[1]), fmaxf(wgt[2], wgt[3]));
-  __syncthreads();
+  m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
   const float f = (t < nsplit && ms != -INFINITY) ? __expf(ms - m) : 0.0f;
-  if (t < nsplit) wgt[t] = f;
   float fl = f * ls;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) fl += __shfl_xor_sync(0xFFFFFFFFu, fl, off);
-  if (t == 0) ml[0] = 0.0f;
+  if (lane == 0) red[4 + warp] = fl;
+  if (t < nsplit) wgt[t] = f;
   __syncthreads();
-  if ((t & 31) == 0) atomicAdd(&ml[0], fl);
-  __syncthreads();
-  const float l = ml[0];
+  const float l = (red[4] + red[5]) + (red[6] + red[7]);
   float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  if (m != -INFINITY) {
-    const float4* src = reinterpret_cast<const float4*>(part_o + (p0 * HQ + h) * D) + t;
-    const int64_t stride = static_cast<int64_t>(HQ) * D / 4;  // float4 between splits
-    for (int s0 = 0; s0 < nsplit; s0 += 8) {
-      float4 v[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        v[j] = s0 + j < nsplit ? __ldg(src + (s0 + j) * stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < kMergeBatch; ++j) {
+    const float fj = j < nsplit ? wgt[j] : 0.0f;
+    acc.x += fj * v[j].x;
+    acc.y += fj * v[j].y;
+    acc.z += fj * v[j].z;
+    acc.w += fj * v[j].w;
+  }
+  for (int s0 = kMergeBatch; s0 < nsplit; s0 += kMergeBatch) {  // more splits than one batch
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float fj = s0 + j < nsplit ? wgt[s0 + j] : 0.0f;
-        acc.x += fj * v[j].x;
-        acc.y += fj * v[j].y;
-        acc.z += fj * v[j].z;
-        acc.w += fj * v[j].w;
-      }
+    for (int j = 0; j < kMergeBatch; ++j)
+      v[j] = s0 + j < nsplit ? __ldg(src + (s0 + j) * stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < kMergeBatch; ++j) {
+      const float fj = s0 + j < nsplit ? wgt[s0 + j] : 0.0f;
+      acc.x += fj * v[j].x;
+      acc.y += fj * v[j].y;
+      acc.z += fj * v[j].z;
+      acc.w += fj * v[j].w;
     }
   }
   const float rl = l > 0.0f ? 1.0f / l : 0.0f;

@@ -73,7 +73,10 @@ def oracle_attend(q, scale, codes, scales, idx, swa, swsc, swa_len):
                          swsc if swa.shape[1] else None, swa_len)
 
 
-@pytest.mark.parametrize("B,n_cap,K,W", [(3, 1024, 100, 70), (2, 4096, 512, 128), (5, 512, 64, 0)])
+# splits per sequence: 4 and 10 (merged inside a thread-block cluster), 1 (no merge), 66 (more
+# than a cluster holds: partials through the workspace and the merge kernel)
+@pytest.mark.parametrize("B,n_cap,K,W", [(3, 1024, 100, 70), (2, 4096, 512, 128), (5, 512, 64, 0),
+                                         (8, 4096, 512, 128), (2, 8192, 4096, 128)])
 def test_attend_matches_oracle(gpu, B, n_cap, K, W):
     dev = gpu
     rng = np.random.default_rng(B * 1000 + K)

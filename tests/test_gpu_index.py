@@ -215,3 +215,39 @@ def test_reindex_with_full_query_recovers_full_topk(gpu):
         assert set(topk[b][topk[b] >= 0]) <= set(pool[b][pool[b] >= 0])
         s, tau = oracle.index_scores(iqb[b], w.numpy()[b], ikb[b, :N[b]], with_tol=True)
         check_selection(topk2[b], topk[b], lambda i: s[i], lambda i: tau[i], f"RI==F b={b}")
+
+
+def _reindex_vs_oracle(iq, w, ik, N, pool, K, gpu, what):
+    B, n_cap = ik.shape[:2]
+    topk2, err = run_reindex(iq, w, ik, N, pool, K, gpu)
+    iqb, ikb = bits(iq).reshape(B, 4, 64), bits(ik).reshape(B, n_cap, 64)
+    ref = oracle.index_reindex(iqb, w.numpy(), ikb, np.asarray(pool, np.int64), K)
+    for b in range(B):
+        s, tau = oracle.index_scores(iqb[b], w.numpy()[b], ikb[b, :N[b]], with_tol=True)
+        ascending_padded(topk2[b], K)
+        check_selection(topk2[b], ref["topk"][b], lambda i: s[i], lambda i: tau[i], f"{what} b={b}")
+    return topk2, err
+
+
+def test_reindex_top_k_concentrated_in_one_stretch_of_the_pool(gpu):
+    """Every Top-K slot lies among the first 600 slots of a 16,384-slot pool."""
+    B, n_cap, K = 2, 16384, 512
+    iq, w, ik = make_case(B, n_cap, seed=51)
+    u = (w[:, :, None] * iq.float()).sum(1)
+    u = u / u.norm(dim=1, keepdim=True)
+    ik = ik.float()
+    ik[:, :600] += 6.0 * u[:, None, :]          # slots 0..599 outscore the rest
+    ik = ik.to(torch.bfloat16)
+    pool = np.tile(np.arange(n_cap, dtype=np.int32), (B, 1))
+    _reindex_vs_oracle(iq, w, ik, [n_cap, n_cap], pool, K, gpu, "one-tile top")
+
+
+@pytest.mark.parametrize("L,K,kind", [(32768, 512, "gauss"), (32768, 4096, "cluster"),
+                                      (700, 512, "gauss"), (5000, 512, "ties")])
+def test_reindex_pool_sizes(gpu, L, K, kind):
+    B, n_cap = 2, 32768
+    iq, w, ik = make_case(B, n_cap, seed=L + K, kind=kind)
+    rng = np.random.default_rng(L)
+    pool = np.stack([np.sort(rng.choice(n_cap, L, replace=False)) for _ in range(B)]).astype(np.int32)
+    pool[:, 5::11] = -1
+    _reindex_vs_oracle(iq, w, ik, [n_cap, n_cap], pool, K, gpu, f"L={L} K={K}")
