@@ -108,6 +108,26 @@ CSA2_API int csa2_append_quant(const void *x, const void *ik, int B, int n, cons
                       float *swa_scale, int W, int32_t *dev_err, csa2_stream_t stream);
 
 /*
+ * CED KV projection with the MXFP4 quantisation in the GEMM epilogue: C = h w^T (bf16 inputs,
+ * fp32 accumulation on the tcgen05 tensor cores), each 16-channel group of a row of C quantised
+ * exactly as csa2_append_quant quantises an appended entry, and the codes and scales written to
+ * the cache rows; the bf16 projection output never reaches memory.
+ * Defines: the CED paragraph of section 一 (the decoder layers' global KV is projected from the
+ * middle layer's hidden state, C_l = H_{L/2} W^KV_l) with the FP4 KV cache paragraph.
+ *   h         bf16 [B, n, d]: hidden states of the n new tokens of each sequence (row-major).
+ *   w         bf16 [512, d]: the layer's KV projection, one row per latent channel (the layout of
+ *             a linear layer's weight).
+ *   d         a multiple of CSA2_CED_D_ALIGN (64), at most CSA2_MAX_CED_D.
+ *   pos, n_cap, codes, scales: as csa2_append_quant (token i of sequence b goes to row pos[b]+i).
+ * Rows outside [0, n_cap) are skipped with CSA2_DEVERR_POS_RANGE. B * n is at most
+ * CSA2_MAX_CED_TOKENS. No workspace; launches one kernel.
+ */
+enum { CSA2_CED_D_ALIGN = 64, CSA2_MAX_CED_D = 65536, CSA2_MAX_CED_TOKENS = 1 << 26 };
+CSA2_API int csa2_ced_project_quant(const void *h, const void *w, int B, int n, int d,
+                                    const int32_t *pos, int n_cap, uint8_t *codes,
+                                    uint8_t *scales, int32_t *dev_err, csa2_stream_t stream);
+
+/*
  * Full-mode indexer: scores every entry, selects the Top-K positions, takes block maxima over
  * 8-position blocks, selects the Top-P blocks and writes the pool.
  * Defines: the hierarchical sparse indexer paragraph of section 一 (Top-512, 2048 blocks x 8).
@@ -190,7 +210,8 @@ enum {
   CSA2_KERNEL_INDEX_SELECT = 2,/* Full-mode candidate collect + final select (two kernels) */
   CSA2_KERNEL_REINDEX = 3,     /* Reindex score + select (two kernels) */
   CSA2_KERNEL_ATTEND = 4,      /* attention + merge (one or two kernels) */
-  CSA2_KERNEL_COUNT = 5
+  CSA2_KERNEL_CED = 5,         /* CED projection with the MXFP4 epilogue */
+  CSA2_KERNEL_COUNT = 6
 };
 CSA2_API int csa2_set_profile_events(int kernel, void *start_event, void *stop_event);
 

@@ -48,6 +48,8 @@ def _declare(L):
     L.oracle_e4m3_encode_array.argtypes = [_P, ctypes.c_int64, _P]
     L.oracle_e2m1_encode_array.argtypes = [_P, ctypes.c_int64, _P]
     L.oracle_mxfp4_quantize_entry.argtypes = [_P, _P, _P]
+    L.oracle_mxfp4_quantize_f32.argtypes = [_P, _P, _P]
+    L.oracle_ced_project.argtypes = [_P, _P, ctypes.c_int64, ctypes.c_int, _P, _P]
     L.oracle_mxfp4_dequantize_entry.argtypes = [_P, _P, _P]
     L.oracle_swa_quantize_token.argtypes = [_P, _P, _P]
     L.oracle_append.restype = ctypes.c_int
@@ -112,6 +114,32 @@ def mxfp4_quantize(x_bf16) -> tuple[np.ndarray, np.ndarray]:
     for i in range(n):
         L.oracle_mxfp4_quantize_entry(_ptr(x[i]), _ptr(codes[i]), _ptr(scales[i]))
     return codes, scales
+
+
+def mxfp4_quantize_f32(x) -> tuple[np.ndarray, np.ndarray]:
+    """fp32 rows [..., 512] -> (codes uint8 [..., 256], scales uint8 [..., 32]); the same
+    definition as mxfp4_quantize, applied to fp32 values (the CED projection output)."""
+    x = _c(x, np.float32)
+    rows = x.reshape(-1, 512)
+    codes = np.zeros((rows.shape[0], 256), np.uint8)
+    scales = np.zeros((rows.shape[0], 32), np.uint8)
+    L = lib()
+    for r in range(rows.shape[0]):
+        L.oracle_mxfp4_quantize_f32(_ptr(rows[r]), _ptr(codes[r]), _ptr(scales[r]))
+    return codes.reshape(x.shape[:-1] + (256,)), scales.reshape(x.shape[:-1] + (32,))
+
+
+def ced_project(h_bits, w_bits):
+    """CED KV projection C = h w^T in double [T1 CED paragraph]. h_bits uint16 (bf16 bits)
+    [M, d], w_bits uint16 [512, d] -> (C float64 [M, 512], sum |h w| float64 [M, 512])."""
+    h = _c(h_bits, np.uint16)
+    w = _c(w_bits, np.uint16)
+    M, d = h.shape
+    assert w.shape == (512, d)
+    c = np.zeros((M, 512), np.float64)
+    a = np.zeros((M, 512), np.float64)
+    lib().oracle_ced_project(_ptr(h), _ptr(w), M, d, _ptr(c), _ptr(a))
+    return c, a
 
 
 def mxfp4_dequantize(codes, scales) -> np.ndarray:

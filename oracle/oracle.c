@@ -165,6 +165,33 @@ void oracle_mxfp4_quantize_entry(const uint16_t *x, uint8_t *codes, uint8_t *sca
   }
 }
 
+/* The same quantisation of a 512-channel row given as fp32 values (the CED projection output):
+ * scale = E4M3 RNE-saturating of the fp32 quotient amax / 6, code = E2M1 RNE-saturating of the
+ * fp32 quotient |x| / scale with the sign bit of x, all codes 0 for a zero scale. */
+void oracle_mxfp4_quantize_f32(const float *x, uint8_t *codes, uint8_t *scales) {
+  for (int g = 0; g < CSA2O_D / 16; ++g) {
+    float amax = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+      float a = fabsf(x[16 * g + i]);
+      if (a > amax) amax = a;
+    }
+    float q = amax / 6.0f;
+    uint8_t sc = oracle_e4m3_encode(q);
+    scales[g] = sc;
+    float s = (float)oracle_e4m3_decode(sc); /* every E4M3 value is exact in fp32 */
+    uint8_t c[16];
+    for (int i = 0; i < 16; ++i) {
+      if (s == 0.0f) {
+        c[i] = 0;
+      } else {
+        float r = fabsf(x[16 * g + i]) / s; /* fp32 quotient */
+        c[i] = (uint8_t)(oracle_e2m1_encode(r) | (f32_signbit(x[16 * g + i]) << 3));
+      }
+    }
+    for (int j = 0; j < 8; ++j) codes[8 * g + j] = (uint8_t)(c[2 * j] | (c[2 * j + 1] << 4));
+  }
+}
+
 /* Dequantised channel i of an MXFP4 entry: E2M1 value times the group's E4M3 scale. */
 static double mxfp4_value(const uint8_t *codes, const uint8_t *scales, int i) {
   uint8_t byte = codes[i / 2];
@@ -299,6 +326,30 @@ int oracle_topk(const double *score, const int64_t *index, int64_t n, int k, int
   topk_ascending(items, n, k, out);
   free(items);
   return 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* CED KV projection [T1 CED paragraph]: the decoder layers' global KV is projected from the   */
+/* middle layer's hidden state, C_l = H_{L/2} W^KV_l. Here C[m][j] = sum_k h[m][k] w[j][k]    */
+/* (w holds one row per latent channel), summed in double; absdot[m][j] = sum_k |h w|, the   */
+/* scale of any fp32 accumulation error of the same sum.                                      */
+/* ------------------------------------------------------------------------------------------ */
+void oracle_ced_project(const uint16_t *h, const uint16_t *w, int64_t M, int d, double *c,
+                        double *absdot) {
+  for (int64_t m = 0; m < M; ++m) {
+    const uint16_t *hr = h + m * d;
+    for (int j = 0; j < CSA2O_D; ++j) {
+      const uint16_t *wr = w + (int64_t)j * d;
+      double acc = 0.0, aacc = 0.0;
+      for (int k = 0; k < d; ++k) {
+        double p = (double)bf16_to_f32(hr[k]) * (double)bf16_to_f32(wr[k]);
+        acc += p;
+        aacc += fabs(p);
+      }
+      c[m * CSA2O_D + j] = acc;
+      if (absdot) absdot[m * CSA2O_D + j] = aacc;
+    }
+  }
 }
 
 /* ------------------------------------------------------------------------------------------ */

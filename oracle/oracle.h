@@ -19,6 +19,9 @@ uint8_t oracle_e4m3_encode(float v);
 void oracle_e4m3_encode_array(const float *v, int64_t n, uint8_t *out);
 void oracle_e2m1_encode_array(const float *v, int64_t n, uint8_t *out);
 
+void oracle_mxfp4_quantize_f32(const float *x, uint8_t *codes, uint8_t *scales);
+void oracle_ced_project(const uint16_t *h, const uint16_t *w, int64_t M, int d, double *c,
+                        double *absdot);
 void oracle_mxfp4_quantize_entry(const uint16_t *x, uint8_t *codes, uint8_t *scales);
 void oracle_mxfp4_dequantize_entry(const uint8_t *codes, const uint8_t *scales, double *out);
 void oracle_swa_quantize_token(const uint16_t *x, uint8_t *e, float *scale);

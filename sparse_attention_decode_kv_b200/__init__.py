@@ -43,6 +43,7 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         L.csa2_append_quant.argtypes = [P, P, I, I, P, I, P, P, P, P, P, I, P, P]
+        L.csa2_ced_project_quant.argtypes = [P, P, I, I, I, P, I, P, P, P, P]
         L.csa2_index_full_workspace_bytes.argtypes = [I, I, I, I]
         L.csa2_index_full_workspace_bytes.restype = Z
         L.csa2_index_full.argtypes = [P, P, P, P, I, I, I, I, P, P, P, Z, P, P]
@@ -112,6 +113,22 @@ def append_quant(x, ik, pos, codes, scales, ik_cache, swa=None, swa_scale=None, 
         _ptr(swa, torch.uint8, "swa"), _ptr(swa_scale, torch.float32, "swa_scale"), W,
         _ptr(dev_err, torch.int32, "dev_err"), _stream(stream))
     _check("csa2_append_quant", st)
+
+
+def ced_project_quant(h, w, pos, codes, scales, dev_err=None, stream=None) -> None:
+    """CED KV projection C = h w^T with the MXFP4 quantisation fused into the GEMM epilogue.
+    h bf16 [B,n,d]; w bf16 [512,d]; pos int32 [B]; codes uint8 [B,n_cap,256];
+    scales uint8 [B,n_cap,32] (token i of sequence b goes to row pos[b] + i)."""
+    B, n, d = h.shape
+    if tuple(w.shape) != (D, d):
+        raise ValueError(f"w must be [{D}, {d}], got {tuple(w.shape)}")
+    n_cap = codes.shape[1]
+    st = lib().csa2_ced_project_quant(
+        _ptr(h, torch.bfloat16, "h"), _ptr(w, torch.bfloat16, "w"), B, n, d,
+        _ptr(pos, torch.int32, "pos"), n_cap, _ptr(codes, torch.uint8, "codes"),
+        _ptr(scales, torch.uint8, "scales"), _ptr(dev_err, torch.int32, "dev_err"),
+        _stream(stream))
+    _check("csa2_ced_project_quant", st)
 
 
 def index_full_workspace_bytes(B: int, n_cap: int, K: int, P: int) -> int:

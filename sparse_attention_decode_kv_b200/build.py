@@ -10,8 +10,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libcsa2.so")
-SOURCES = ["abi.cu", "append.cu", "attend.cu", "index.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "internal.h", "select.cuh"]
+SOURCES = ["abi.cu", "append.cu", "attend.cu", "ced.cu", "index.cu", "noalloc.cu"]
+HEADERS = ["common.cuh", "internal.h", "select.cuh", "tcgen05.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

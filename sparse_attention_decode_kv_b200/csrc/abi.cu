@@ -26,6 +26,19 @@ void profile_end(int kernel, cudaStream_t s) {
   if (g_prof_stop[kernel] != nullptr) cudaEventRecord(g_prof_stop[kernel], s);
 }
 
+TensorMapEncodeFn tensor_map_encoder() {
+  static std::once_flag once;
+  static TensorMapEncodeFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<TensorMapEncodeFn>(p);
+  });
+  return fn;
+}
+
 int device_sm_count() {
   static std::mutex mu;
   static std::vector<int> cache;
@@ -60,7 +73,7 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CU
 
 extern "C" {
 
-int csa2_abi_version(void) { return 1; }
+int csa2_abi_version(void) { return 2; }
 
 uint64_t csa2_launch_count(void) { return csa2::g_launches.load(); }
 
@@ -101,6 +114,22 @@ int csa2_append_quant(const void* x, const void* ik, int B, int n, const int32_t
   return cuda_status(csa2::launch_append(x, ik, B, n, pos, n_cap, codes, scales, ik_cache, swa,
                                          swa_scale, W, dev_err,
                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int csa2_ced_project_quant(const void* h, const void* w, int B, int n, int d, const int32_t* pos,
+                           int n_cap, uint8_t* codes, uint8_t* scales, int32_t* dev_err,
+                           csa2_stream_t stream) {
+  if (B <= 0 || n < 0 || n_cap <= 0 || (n_cap % CSA2_S) != 0) return CSA2_ERR_INVALID;
+  if (d < CSA2_CED_D_ALIGN || (d % CSA2_CED_D_ALIGN) != 0) return CSA2_ERR_INVALID;
+  if (B > CSA2_MAX_B || n_cap > CSA2_MAX_NCAP || d > CSA2_MAX_CED_D ||
+      static_cast<int64_t>(B) * n > CSA2_MAX_CED_TOKENS)
+    return CSA2_ERR_UNSUPPORTED;
+  if (!ptr_ok(h) || !ptr_ok(w) || !ptr_ok(pos) || !ptr_ok(codes) || !ptr_ok(scales))
+    return CSA2_ERR_INVALID;
+  if (dev_err != nullptr && (reinterpret_cast<uintptr_t>(dev_err) & 3u)) return CSA2_ERR_INVALID;
+  if (n == 0) return CSA2_OK;
+  return cuda_status(csa2::launch_ced_quant(h, w, B, n, d, pos, n_cap, codes, scales, dev_err,
+                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t csa2_index_full_workspace_bytes(int B, int n_cap, int K, int P) {

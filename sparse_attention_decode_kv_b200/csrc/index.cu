@@ -751,25 +751,6 @@ FullLayout full_layout(int B, int n_cap) {
   return l;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static std::once_flag once;
-  static EncodeTiledFn fn = nullptr;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
 template <class Kern>
 cudaError_t set_smem(Kern k, size_t bytes, std::vector<int>& done) {
   int dev = 0;
@@ -804,7 +785,7 @@ cudaError_t launch_index_full(const void* iq, const float* w, const void* ik_cac
   uint32_t* ccnt = reinterpret_cast<uint32_t*>(base + l.ccnt);
   uint64_t* cand = reinterpret_cast<uint64_t*>(base + l.cand);
 
-  EncodeTiledFn enc = encode_fn();
+  const TensorMapEncodeFn enc = tensor_map_encoder();
   if (enc == nullptr) return cudaErrorNotSupported;
   CUtensorMap map;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(DI), static_cast<cuuint64_t>(n_cap),

@@ -1,6 +1,7 @@
 // internal.h -- host-side launchers behind the C ABI (not part of the public interface).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -11,6 +12,13 @@ void count_launches(int n);   // adds to the process-wide launch counter
 void profile_begin(int kernel, cudaStream_t s);  // records the start event if one is set
 void profile_end(int kernel, cudaStream_t s);    // records the stop event if one is set
 int device_sm_count();        // SMs of the current device (cached per device)
+
+// cuTensorMapEncodeTiled from the driver (looked up once through the runtime), or null.
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                      const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                      const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                      CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+TensorMapEncodeFn tensor_map_encoder();
 
 // Quantize-on-append; one warp per new entry.
 cudaError_t launch_append(const void* x, const void* ik, int B, int n, const int32_t* pos,
@@ -39,5 +47,10 @@ cudaError_t launch_index_reindex(const void* iq, const float* w, const void* ik_
                                  const int32_t* N, int B, int n_cap, const int32_t* pool, int L,
                                  int K, int32_t* topk, void* ws, int32_t* dev_err,
                                  cudaStream_t s);
+
+// CED KV projection with the MXFP4 quantisation in the GEMM epilogue (tcgen05).
+cudaError_t launch_ced_quant(const void* h, const void* w, int B, int n, int d, const int32_t* pos,
+                             int n_cap, uint8_t* codes, uint8_t* scales, int32_t* dev_err,
+                             cudaStream_t s);
 
 }  // namespace csa2

@@ -1,0 +1,114 @@
+// tcgen05.cuh -- thin wrappers over the sm_100a tensor-core (tcgen05) and TMA instructions used
+// by the GEMM kernels: tensor-memory allocation, shared-memory matrix descriptors, the MMA issue,
+// its completion commit, tensor-memory loads and the fences that order them with thread barriers.
+//
+// Encodings follow the PTX ISA for sm_100a: a shared-memory matrix descriptor holds the start
+// address (bits 0-13), the leading and stride byte offsets (bits 16-29, 32-45; 16-byte units),
+// the descriptor version 1 (bits 46-47) and the swizzle mode (bits 61-63; 2 = 128-byte swizzle);
+// the kind::f16 instruction descriptor holds the accumulator type (bits 4-5), the A and B types
+// (bits 7-9, 10-12), their major-ness (bits 15, 16), N / 8 (bits 17-22) and M / 16 (bits 24-28).
+#pragma once
+
+#include "common.cuh"
+
+namespace csa2 {
+
+// ------------------------------------------------------------------------------ TMEM allocation
+
+// Allocate `ncols` tensor-memory columns (a power of two >= 32) for this CTA; the base address is
+// written to *dst (shared memory). Whole warp.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+// Whole warp; every tensor-memory access of the CTA must have completed.
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tcgen05_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tcgen05_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// --------------------------------------------------------------------------------- descriptors
+
+// K-major operand tile in shared memory, rows of 128 bytes (64 bf16) written by a TMA copy with
+// 128-byte swizzle; consecutive 8-row groups 1024 bytes apart. `addr` is the shared address of
+// the K-slice (the tile base, 1024-byte aligned, plus 32 bytes per 16 K elements).
+__device__ __forceinline__ uint64_t umma_desc_k128(uint32_t addr) {
+  uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;    // leading byte offset (unused for swizzled K-major)
+  d |= static_cast<uint64_t>(64u) << 32;   // stride byte offset: 1024 bytes
+  d |= static_cast<uint64_t>(1u) << 46;    // descriptor version
+  d |= static_cast<uint64_t>(2u) << 61;    // 128-byte swizzle
+  return d;
+}
+
+// kind::f16 instruction descriptor: bf16 A and B (both K-major), fp32 accumulator, M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// ----------------------------------------------------------------------------------------- MMA
+
+// D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on `bar` when every MMA this thread issued before has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// ------------------------------------------------------------------------------------ TMEM load
+
+// 16 consecutive 32-bit columns of this warp's 32 lanes (lane i of the warp reads lane
+// quarter_base + i); complete only after tmem_wait_ld().
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ----------------------------------------------------------------------------------------- TMA
+
+// 2-D tiled bulk tensor load into this CTA's shared memory, completing on `bar` (no multicast).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                            int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+}  // namespace csa2

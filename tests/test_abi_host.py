@@ -43,7 +43,7 @@ def test_status_strings_and_version(L):
     assert csa2.status_string(0) == "CSA2_OK"
     for s in (-1, -2, -3, -4, -5, -6):
         assert csa2.status_string(s).startswith("CSA2_ERR")
-    assert L.csa2_abi_version() == 1
+    assert L.csa2_abi_version() == 2
     assert csa2.launch_count() >= 0
 
 
@@ -84,6 +84,30 @@ def test_append_rejects_bad_arguments(L):
     assert append(L, B=5000) == UNSUPPORTED
     assert append(L, W=5000) == UNSUPPORTED
     assert append(L, n=0) == OK                      # nothing to do: no launch
+
+
+def ced(L, **kw):
+    a = dict(h=FAKE, w=FAKE, B=2, n=100, d=256, pos=FAKE, n_cap=64, codes=FAKE, scales=FAKE,
+             dev_err=None)
+    a.update(kw)
+    return L.csa2_ced_project_quant(P(a["h"]), P(a["w"]), a["B"], a["n"], a["d"], P(a["pos"]),
+                                    a["n_cap"], P(a["codes"]), P(a["scales"]), P(a["dev_err"]),
+                                    None)
+
+
+def test_ced_projection_rejects_bad_arguments(L):
+    assert ced(L, B=0) == INVALID
+    assert ced(L, n=-1) == INVALID
+    assert ced(L, d=0) == INVALID
+    assert ced(L, d=100) == INVALID                  # not a multiple of 64
+    assert ced(L, n_cap=60) == INVALID
+    assert ced(L, h=0) == INVALID
+    assert ced(L, w=MIS) == INVALID
+    assert ced(L, scales=0) == INVALID
+    assert ced(L, dev_err=FAKE + 2) == INVALID
+    assert ced(L, d=65600) == UNSUPPORTED
+    assert ced(L, B=4096, n=1 << 15) == UNSUPPORTED  # more than 2^26 tokens
+    assert ced(L, n=0) == OK                         # nothing to do: no launch
 
 
 def index_full(L, ws_bytes=None, **kw):
