@@ -9,6 +9,11 @@ layer-step = one layer's decode step for the whole batch) and achieved HBM GB/s 
 algorithmic bytes (indexer keys read + gathered MXFP4 codes and scales + FP8 SWA rows).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+  python bench.py --ced [--steps K] [--warmup W]
+
+--ced measures the CED KV projection with the MXFP4 epilogue instead (8 x 4,096 new tokens,
+hidden size 4,096: a tensor-core-bound GEMM), reported in TFLOP/s against the measured bf16
+tensor peak.
 
 With --gpus N > 1 run under torchrun: every rank decodes its own batch (data parallel, no
 collective on the data path); the step time is the max over ranks.
@@ -53,6 +58,8 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ced", action="store_true",
+                    help="measure the CED KV projection with the MXFP4 epilogue instead")
     ap.add_argument("--breakdown", action="store_true",
                     help="also time each library call of the step (eager, synchronised)")
     return ap.parse_args()
@@ -64,6 +71,14 @@ def measured_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 def scan_traffic_per_launch(wl):
@@ -606,11 +621,132 @@ def run_reference(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+
+# ------------------------------------------------------------------ CED projection measurement
+
+CED_METRIC = "CED KV projection + MXFP4 epilogue TFLOP/s (bf16 tensor cores), 1 B200"
+CED_SHAPE = dict(B=8, n=4096, d=4096)   # 32,768 new tokens, hidden size 4,096
+
+
+def ced_cpu_baseline(h, w, rows=8):
+    """The oracle's projection and quantisation of a few rows, scaled to TFLOP/s."""
+    import numpy as np
+    import oracle
+    from oracle import build as oracle_build
+    oracle_build.build()
+    d = h.shape[-1]
+    hb = h.reshape(-1, d)[:rows].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    wb = w.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    t = time.perf_counter()
+    c, _ = oracle.ced_project(hb, wb)
+    oracle.mxfp4_quantize_f32(c.astype(np.float32))
+    sec = time.perf_counter() - t
+    value = 2.0 * rows * 512 * d / sec / 1e12
+    return {"value": round(value, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} token rows of d = {d} projected and quantised ({sec:.2f} s)",
+            "seconds": round(sec, 2)}
+
+
+def run_ced(args, world, rank, local):
+    import sparse_attention_decode_kv_b200 as csa2
+    from sparse_attention_decode_kv_b200 import build as csa2_build
+    if rank == 0:
+        csa2_build.build()
+    barrier(world)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    B, n, d = CED_SHAPE["B"], CED_SHAPE["n"], CED_SHAPE["d"]
+    g = torch.Generator(device=dev).manual_seed(1000 + rank)
+    h = torch.randn(B, n, d, device=dev, generator=g).to(torch.bfloat16)
+    w = (torch.randn(512, d, device=dev, generator=g) / d ** 0.5).to(torch.bfloat16)
+    codes = torch.empty(B, n, 256, dtype=torch.uint8, device=dev)
+    scales = torch.empty(B, n, 32, dtype=torch.uint8, device=dev)
+    pos = torch.zeros(B, dtype=torch.int32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        csa2.ced_project_quant(h, w, pos, codes, scales, err)
+
+    K, W = args.steps, args.warmup
+    launches0 = csa2.launch_count()
+    step()
+    torch.cuda.synchronize()
+    per_step_launches = csa2.launch_count() - launches0
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(K):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = max_over_ranks(world, t0.elapsed_time(t1), dev) / K
+    if int(err.item()):
+        raise RuntimeError(f"device error flags {int(err.item()):#x} during the benchmark")
+    flop = 2.0 * B * n * 512 * d
+    tflops = flop / (ms / 1e3) / 1e12
+    peak, peak_kind = measured_tensor_peak()
+
+    e2e = None
+    if not args.no_e2e:
+        hh = h.cpu().pin_memory()
+        hc = torch.empty(codes.shape, dtype=torch.uint8).pin_memory()
+        hs = torch.empty(scales.shape, dtype=torch.uint8).pin_memory()
+        ke = max(1, min(K, 20))
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(ke):
+            h.copy_(hh, non_blocking=True)
+            step()
+            hc.copy_(codes, non_blocking=True)
+            hs.copy_(scales, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / ke
+        e2e = {"value": round(flop / (e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h.numel() * 2,
+               "d2h_bytes_per_step": codes.numel() + scales.numel()}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = ced_cpu_baseline(h, w)
+    line = {
+        "metric": CED_METRIC, "value": round(world * tflops, 2), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16-in fp32-acc (mxfp4 out)", "data": "synthetic",
+        "config": {"workload": f"ced-projection-B{B}-n{n}-d{d}", "tokens_per_gpu": B * n,
+                   "d": d, "channels": 512,
+                   "l2": "inputs larger than L2 (h is %.0f MB)" % (h.numel() * 2 / 1e6),
+                   "parallelism": f"dp{world} (independent token batches)"},
+        "roofline": {"kernel": "ced_quant_kernel (tcgen05 GEMM + MXFP4 epilogue)",
+                     "bound": "tensor", "achieved": round(tflops, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "peak_kind": peak_kind,
+                     "algorithmic_flop_per_launch": flop, "launch_ms": round(ms, 4),
+                     "traffic": None},
+        "gpu_launches": per_step_launches * K,
+        "clocks": clocks.summary(),
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
 def main():
     args = parse()
     world, rank, local = dist_setup()
     try:
-        if args.impl == "reference":
+        if args.ced and args.impl == "ours":
+            run_ced(args, world, rank, local)
+        elif args.impl == "reference":
             run_reference(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
