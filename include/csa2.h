@@ -65,7 +65,9 @@ enum {
   CSA2_MAX_K = 4096,       /* Top-K of the indexers; indices per sequence for attention */
   CSA2_MAX_P = 4096,       /* pool blocks */
   CSA2_MAX_POOL = 32768,   /* pool slots scored by a Reindex call */
-  CSA2_MAX_W = 4096,       /* SWA ring length */
+  CSA2_MAX_W = 4096,       /* SWA ring length; SWA rows one query attends to */
+  CSA2_MAX_QUERIES = 1 << 20,   /* queries of one csa2_attend_queries call */
+  CSA2_MAX_SWA_ROWS = 1 << 24,  /* rows per sequence of the SWA buffer of csa2_attend_queries */
   CSA2_MAX_NCAP = 1 << 28  /* rows per sequence */
 };
 
@@ -196,6 +198,32 @@ CSA2_API int csa2_attend(int mode, const void *q, float softmax_scale, const uin
                 const uint8_t *swa, const float *swa_scale, const int32_t *swa_len, int W, int B,
                 float *out, float *lse, void *ws, size_t ws_bytes, int32_t *dev_err,
                 csa2_stream_t stream);
+
+/*
+ * Sparse attention of many queries per sequence (prefill, or verification of several drafted
+ * tokens): query b reads the cache of sequence qseq[b], its own K indices idx[b] and the SWA
+ * rows swa_lo[b] .. swa_lo[b] + swa_len[b] - 1 of that sequence's FP8 buffer; otherwise the same
+ * computation as csa2_attend (which is the case of one query per sequence and the ring).
+ * Defines: the Reuse mode of section 一 in prefill (each prompt token's layer attends to its own
+ * selected entries plus its sliding window) and the 15-kernel prefill flow of section 二.
+ *   q         bf16 [Q, 16, 512]; out float [Q, 16, 512]; lse float [Q, 16] or NULL.
+ *   codes, scales, N: B cache sequences as for csa2_attend.
+ *   qseq      int32 [Q] (device): sequence of each query; entries outside [0, B) give an empty
+ *             query and CSA2_DEVERR_INDEX_RANGE.
+ *   idx       int32 [Q, K]: entry positions of each query, -1 = none.
+ *   swa       uint8 [B, S, 512] E4M3 rows and swa_scale float [B, S] (fp32 per-row scales);
+ *             swa_lo, swa_len int32 [Q] (device): the query's rows, 0 <= swa_len <= W <= S
+ *             (out-of-range windows are clamped and flagged with CSA2_DEVERR_NLEN). W = 0: no
+ *             SWA rows, and swa, swa_scale, swa_lo, swa_len may be NULL.
+ *   ws        csa2_attend_workspace_bytes(Q, K, W) bytes.
+ */
+CSA2_API int csa2_attend_queries(const void *q, float softmax_scale, const uint8_t *codes,
+                                 const uint8_t *scales, int B, int n_cap, const int32_t *N,
+                                 const int32_t *qseq, const int32_t *idx, int K,
+                                 const uint8_t *swa, const float *swa_scale, int S,
+                                 const int32_t *swa_lo, const int32_t *swa_len, int W, int Q,
+                                 float *out, float *lse, void *ws, size_t ws_bytes,
+                                 int32_t *dev_err, csa2_stream_t stream);
 
 /*
  * Profiling hook (no counterpart on the pages): when events are set for a kernel id, every later

@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
         L.csa2_attend_workspace_bytes.restype = Z
         L.csa2_attend.argtypes = [I, P, ctypes.c_float, P, P, I, P, P, I, P, P, P, I, I, P, P, P,
                                   Z, P, P]
+        L.csa2_attend_queries.argtypes = [P, ctypes.c_float, P, P, I, I, P, P, P, I, P, P, I, P, P,
+                                          I, I, P, P, P, Z, P, P]
         L.csa2_status_string.argtypes = [I]
         L.csa2_status_string.restype = ctypes.c_char_p
         L.csa2_launch_count.restype = ctypes.c_uint64
@@ -201,6 +203,28 @@ def attend(mode, q, softmax_scale, codes, scales, N, idx, swa, swa_scale, swa_le
         _ptr(lse, torch.float32, "lse"), ws_ptr, ws_bytes, _ptr(dev_err, torch.int32, "dev_err"),
         _stream(stream))
     _check("csa2_attend", st)
+
+
+def attend_queries(q, softmax_scale, codes, scales, N, qseq, idx, swa, swa_scale, swa_lo, swa_len,
+                   W, out, lse, ws, dev_err=None, stream=None) -> None:
+    """Sparse attention of many queries per sequence. q bf16 [Q,16,512]; codes/scales of B
+    sequences; N int32 [B]; qseq int32 [Q] (each query's sequence); idx int32 [Q,K];
+    swa uint8 [B,S,512] / swa_scale f32 [B,S] / swa_lo, swa_len int32 [Q] (the query's SWA rows,
+    swa_len <= W), or all None with W = 0; out f32 [Q,16,512]; lse f32 [Q,16] or None."""
+    Q, K = idx.shape
+    B, n_cap = codes.shape[0], codes.shape[1]
+    S = 0 if swa is None else swa.shape[1]
+    ws_ptr = _ptr(ws, None, "ws") if ws is not None and ws.numel() > 0 else None
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    st = lib().csa2_attend_queries(
+        _ptr(q, torch.bfloat16, "q"), float(softmax_scale), _ptr(codes, torch.uint8, "codes"),
+        _ptr(scales, torch.uint8, "scales"), B, n_cap, _ptr(N, torch.int32, "N"),
+        _ptr(qseq, torch.int32, "qseq"), _ptr(idx, torch.int32, "idx"), K,
+        _ptr(swa, torch.uint8, "swa"), _ptr(swa_scale, torch.float32, "swa_scale"), S,
+        _ptr(swa_lo, torch.int32, "swa_lo"), _ptr(swa_len, torch.int32, "swa_len"), int(W), Q,
+        _ptr(out, torch.float32, "out"), _ptr(lse, torch.float32, "lse"), ws_ptr, ws_bytes,
+        _ptr(dev_err, torch.int32, "dev_err"), _stream(stream))
+    _check("csa2_attend_queries", st)
 
 
 # ------------------------------------------------------------------------------- buffer helpers

@@ -198,7 +198,37 @@ int csa2_attend(int mode, const void* q, float softmax_scale, const uint8_t* cod
   if (need > 0 && (ws == nullptr || !aligned16(ws) || ws_bytes < need)) return CSA2_ERR_WORKSPACE;
   return cuda_status(csa2::launch_attend(q, softmax_scale, codes, scales, n_cap, N, idx, K,
                                          W > 0 ? swa : nullptr, W > 0 ? swa_scale : nullptr,
-                                         W > 0 ? swa_len : nullptr, W, B, out, lse, ws, dev_err,
+                                         W > 0 ? swa_len : nullptr, W, nullptr, nullptr, W, B, B,
+                                         out, lse, ws, dev_err,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int csa2_attend_queries(const void* q, float softmax_scale, const uint8_t* codes,
+                        const uint8_t* scales, int B, int n_cap, const int32_t* N,
+                        const int32_t* qseq, const int32_t* idx, int K, const uint8_t* swa,
+                        const float* swa_scale, int S, const int32_t* swa_lo,
+                        const int32_t* swa_len, int W, int Q, float* out, float* lse, void* ws,
+                        size_t ws_bytes, int32_t* dev_err, csa2_stream_t stream) {
+  if (Q <= 0 || B <= 0 || n_cap <= 0 || (n_cap % CSA2_S) != 0 || K <= 0 || W < 0 || S < 0)
+    return CSA2_ERR_INVALID;
+  if (W > S) return CSA2_ERR_INVALID;  // a window never holds more rows than the buffer
+  if (Q > CSA2_MAX_QUERIES || B > CSA2_MAX_B || n_cap > CSA2_MAX_NCAP || K > CSA2_MAX_K ||
+      W > CSA2_MAX_W || S > CSA2_MAX_SWA_ROWS)
+    return CSA2_ERR_UNSUPPORTED;
+  if (!(softmax_scale == softmax_scale)) return CSA2_ERR_INVALID;  // NaN
+  if (!ptr_ok(q) || !ptr_ok(codes) || !ptr_ok(scales) || !ptr_ok(N) || !ptr_ok(qseq) ||
+      !ptr_ok(idx) || !ptr_ok(out) || !ptr_ok(lse, true))
+    return CSA2_ERR_INVALID;
+  if (W > 0 && (!ptr_ok(swa) || !ptr_ok(swa_scale) || !ptr_ok(swa_lo) || !ptr_ok(swa_len)))
+    return CSA2_ERR_INVALID;
+  if (dev_err != nullptr && (reinterpret_cast<uintptr_t>(dev_err) & 3u)) return CSA2_ERR_INVALID;
+  const size_t need = csa2::attend_workspace_bytes(Q, K, W);
+  if (need > 0 && (ws == nullptr || !aligned16(ws) || ws_bytes < need)) return CSA2_ERR_WORKSPACE;
+  // the kernels check every qseq entry against B (a bad one gives an empty query and a flag)
+  return cuda_status(csa2::launch_attend(q, softmax_scale, codes, scales, n_cap, N, idx, K,
+                                         W > 0 ? swa : nullptr, W > 0 ? swa_scale : nullptr,
+                                         W > 0 ? swa_len : nullptr, W, qseq,
+                                         W > 0 ? swa_lo : nullptr, S, B, Q, out, lse, ws, dev_err,
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -6,6 +6,12 @@
 // Reading: K = V = the dequantised entry; z = softmax_scale * q . v over the selected entries and
 // the valid SWA slots together; out = sum softmax(z) v; lse = log sum exp(z).
 //
+// Queries: in a decode step query b belongs to cache sequence b and its SWA rows are slots
+// 0 .. swa_len[b]-1 of sequence b's ring. The multi-query form (prefill or verification of
+// several tokens per sequence) maps query b to cache sequence qseq[b] and to rows swa_lo[b] ..
+// swa_lo[b] + swa_len[b] - 1 of that sequence's FP8 SWA buffer of S rows; b below always names
+// the query.
+//
 // Work split: the K index slots and the W SWA slots are cut into tiles of 64 items (index tiles
 // and SWA tiles never mix); grid = (splits, B) and each CTA runs an online softmax over a
 // contiguous run of tiles. With one split the CTA writes the result; otherwise it writes an
@@ -70,7 +76,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                   const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                   int n_cap, const int32_t* __restrict__ N, const int32_t* __restrict__ idx, int K,
                   const uint8_t* __restrict__ swa, const float* __restrict__ swa_scale,
-                  const int32_t* __restrict__ swa_len, int W, float* __restrict__ out,
+                  const int32_t* __restrict__ swa_len, int W, const int32_t* __restrict__ qseq,
+                  const int32_t* __restrict__ swa_lo, int S, int nseq, float* __restrict__ out,
                   float* __restrict__ lse, float* __restrict__ part_o,
                   float* __restrict__ part_ml, int32_t* dev_err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -87,17 +94,33 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int t_begin = static_cast<int>(static_cast<int64_t>(split) * tiles / nsplit);
   const int t_end = static_cast<int>(static_cast<int64_t>(split + 1) * tiles / nsplit);
 
-  int nb = __ldg(N + b);
+  int sb = qseq ? __ldg(qseq + b) : b;  // cache sequence of query b
+  const bool sb_ok = sb >= 0 && sb < nseq;
+  if (!sb_ok) {  // an unknown sequence: the query attends to nothing
+    if (tid == 0) flag_error(dev_err, CSA2_DEVERR_INDEX_RANGE);
+    sb = 0;
+  }
+  int nb = sb_ok ? __ldg(N + sb) : 0;
   if (nb < 0 || nb > n_cap) {
     if (tid == 0) flag_error(dev_err, CSA2_DEVERR_NLEN);
     nb = max(0, min(nb, n_cap));
   }
   int sl = 0;
   if (W > 0) {
-    sl = swa_len ? __ldg(swa_len + b) : 0;
+    sl = (swa_len && sb_ok) ? __ldg(swa_len + b) : 0;
     if (sl < 0 || sl > W) {
       if (tid == 0) flag_error(dev_err, CSA2_DEVERR_NLEN);
       sl = max(0, min(sl, W));
+    }
+  }
+  // first SWA row of this query in its sequence's buffer of S rows (the ring: 0, S = W)
+  int slo = 0;
+  if (swa_lo != nullptr && sl > 0) {
+    slo = __ldg(swa_lo + b);
+    if (slo < 0 || slo + sl > S) {
+      if (tid == 0) flag_error(dev_err, CSA2_DEVERR_NLEN);
+      slo = max(0, min(slo, S));
+      sl = min(sl, S - slo);
     }
   }
 
@@ -156,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
 
   const uint32_t q_base = smem_u32(sm.q), v_base = smem_u32(sm.v), p_base = smem_u32(sm.p);
-  const int64_t seq_row0 = static_cast<int64_t>(b) * n_cap;
+  const int64_t seq_row0 = static_cast<int64_t>(sb) * n_cap;
 
   for (int tile = t_begin; tile < t_end; ++tile) {
     const bool is_swa = tile >= tiles_idx;
@@ -216,10 +239,11 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int item = pass * 16 + (tid >> 4);
           const int slot = base + item;
           const bool valid = item < count && slot < sl;
-          const uint8_t* rowp = swa + (static_cast<int64_t>(b) * W + (valid ? slot : 0)) * D + 32 * r;
+          const int64_t srow = static_cast<int64_t>(sb) * S + slo + (valid ? slot : 0);
+          const uint8_t* rowp = swa + srow * D + 32 * r;
           e[pass][0] = valid ? ldg_nc_v4(rowp) : make_uint4(0u, 0u, 0u, 0u);
           e[pass][1] = valid ? ldg_nc_v4(rowp + 16) : make_uint4(0u, 0u, 0u, 0u);
-          iscale[pass] = valid ? __ldg(swa_scale + static_cast<int64_t>(b) * W + slot) : 1.0f;
+          iscale[pass] = valid ? __ldg(swa_scale + srow) : 1.0f;
         }
 #pragma unroll
         for (int pass = 0; pass < 4; ++pass) {
@@ -491,8 +515,9 @@ size_t attend_workspace_bytes(int B, int K, int W) {
 cudaError_t launch_attend(const void* q, float softmax_scale, const uint8_t* codes,
                           const uint8_t* scales, int n_cap, const int32_t* N, const int32_t* idx,
                           int K, const uint8_t* swa, const float* swa_scale,
-                          const int32_t* swa_len, int W, int B, float* out, float* lse, void* ws,
-                          int32_t* dev_err, cudaStream_t s) {
+                          const int32_t* swa_len, int W, const int32_t* qseq,
+                          const int32_t* swa_lo, int S, int nseq, int B, float* out, float* lse,
+                          void* ws, int32_t* dev_err, cudaStream_t s) {
   const int splits = attend_split_count(B, K, W);
   float* part_o = nullptr;
   float* part_ml = nullptr;
@@ -513,7 +538,8 @@ cudaError_t launch_attend(const void* q, float softmax_scale, const uint8_t* cod
   profile_begin(CSA2_KERNEL_ATTEND, s);
   cudaError_t e = launch_pdl(attend_kernel, dim3(splits, B), dim3(kThreads), smem, s,
                              static_cast<const uint16_t*>(q), softmax_scale, codes, scales, n_cap,
-                             N, idx, K, swa, swa_scale, swa_len, W, out, lse, part_o, part_ml,
+                             N, idx, K, swa, swa_scale, swa_len, W, qseq, swa_lo, S, nseq, out,
+                             lse, part_o, part_ml,
                              dev_err);
   count_launches(1);
   if (e == cudaSuccess) e = cudaGetLastError();
