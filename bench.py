@@ -628,7 +628,7 @@ CED_METRIC = "CED KV projection + MXFP4 epilogue TFLOP/s (bf16 tensor cores), 1 
 CED_SHAPE = dict(B=8, n=4096, d=4096)   # 32,768 new tokens, hidden size 4,096
 
 
-def ced_cpu_baseline(h, w, rows=8):
+def ced_cpu_baseline(h, w, rows=4096):
     """The oracle's projection and quantisation of a few rows, scaled to TFLOP/s."""
     import numpy as np
     import oracle

@@ -13,7 +13,7 @@
 // the query.
 //
 // Work split: the K index slots and the W SWA slots are cut into tiles of 64 items (index tiles
-// and SWA tiles never mix); grid = (splits, B) and each CTA runs an online softmax over a
+// and SWA tiles never mix); grid = (B, splits) and each CTA runs an online softmax over a
 // contiguous run of tiles. With one split the CTA writes the result; otherwise it writes an
 // unnormalised partial (m, l, o) and attend_merge_kernel combines the partials by log-sum-exp.
 //
@@ -39,12 +39,16 @@ constexpr int kTile = 64;
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kTargetCtas = 296;  // 148 SMs x 2 resident CTAs
+constexpr int kRawRow = D / 2 + D / 16;  // 288 bytes: codes then scales of one MXFP4 entry
+constexpr int kZs = kTile + 8;  // partial-logit row stride: the float2 stores of 16 lanes hit 16 bank pairs
 
 struct __align__(16) AttendSmem {
   uint16_t q[HQ * D];        // fp16 [16][512], 16-byte chunks XOR-swizzled by (row & 7)
   uint16_t v[kTile * D];     // fp16 [64][512], same swizzle
+  uint8_t raw[kTile * kRawRow];  // the next MXFP4 tile's rows, fetched during this tile;
+                                 // 16-byte aligned (offset 81920) for the 16-byte copies
   uint16_t p[HQ * kTile];    // fp16 [16][64], same swizzle (8 chunks per row)
-  float zp[2][HQ * kTile];   // partial logits of the current tile over dims 0..255 / 256..511
+  float zp[2][HQ * kZs];     // partial logits of the current tile over dims 0..255 / 256..511
   float item_scale[kTile];   // 1 (MXFP4) or the SWA token's fp32 scale
   int item_valid[kTile];
   float q_unscale[HQ];       // 2^(e_h - 14) * softmax_scale
@@ -52,8 +56,20 @@ struct __align__(16) AttendSmem {
   float tile_pf;             // power of two applied to P on SWA tiles
 };
 
-__device__ __forceinline__ uint32_t swz1024(int row, int chunk) {  // 64 chunks per row
-  return static_cast<uint32_t>(row * 1024 + ((chunk ^ (row & 7)) << 4));
+// 16-byte asynchronous copy global -> shared; src_bytes 0 fills the 16 bytes with zeros.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Row of 64 16-byte chunks. The low three chunk bits are XORed with the row's low bits (the 8 rows
+// of an ldmatrix read at one chunk fall in 8 distinct bank groups) and with the chunk's own bits
+// 3..5 (the chunks 4r + k, r = 0..7, that 8 threads store at once also fall in 8 distinct groups).
+__device__ __forceinline__ uint32_t swz1024(int row, int chunk) {
+  return static_cast<uint32_t>(row * 1024 + ((chunk ^ (row & 7) ^ ((chunk >> 3) & 7)) << 4));
 }
 __device__ __forceinline__ uint32_t swz128(int row, int chunk) {  // 8 chunks per row
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
@@ -84,7 +100,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   AttendSmem& sm = *reinterpret_cast<AttendSmem*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, c = lane & 3;
-  const int b = blockIdx.y, split = blockIdx.x, nsplit = gridDim.x;
+  const int b = blockIdx.x, split = blockIdx.y, nsplit = gridDim.y;  // b on x: up to 2^31 - 1
   pdl_wait();
   pdl_launch_dependents();
 
@@ -181,10 +197,25 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t q_base = smem_u32(sm.q), v_base = smem_u32(sm.v), p_base = smem_u32(sm.p);
   const int64_t seq_row0 = static_cast<int64_t>(sb) * n_cap;
 
+  // Software pipeline over MXFP4 tiles: while a tile is computed, the next one's rows stream
+  // into sm.raw with cp.async (its indices were requested when the tile began), so only the
+  // first tile of a CTA and the SWA tiles wait for their gather.
+  int pos_staged[4] = {-1, -1, -1, -1};  // positions of the tile held in sm.raw
+  bool staged = false;
   for (int tile = t_begin; tile < t_end; ++tile) {
     const bool is_swa = tile >= tiles_idx;
     const int base = is_swa ? (tile - tiles_idx) * kTile : tile * kTile;
     const int count = min(kTile, (is_swa ? W : K) - base);
+    const bool next_mx = tile + 1 < t_end && tile + 1 < tiles_idx;
+    int pos_next[4] = {-1, -1, -1, -1};
+    if (next_mx) {
+#pragma unroll
+      for (int pass = 0; pass < 4; ++pass) {
+        const int item = pass * 16 + (tid >> 4);
+        if (item < min(kTile, K - (base + kTile)))
+          pos_next[pass] = __ldg(idx + static_cast<int64_t>(b) * K + base + kTile + item);
+      }
+    }
 
     // ---- gather + dequantise: 16 threads per item, 32 channels per thread, 4 passes of 16 items.
     // All index loads, then all row loads, then the conversions: two memory round trips.
@@ -196,18 +227,26 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int pass = 0; pass < 4; ++pass) {
           const int item = pass * 16 + (tid >> 4);
-          pos[pass] = tile == t_begin ? pos_first[pass]
+          pos[pass] = staged ? pos_staged[pass]
+                      : tile == t_begin ? pos_first[pass]
                       : (item < count ? __ldg(idx + static_cast<int64_t>(b) * K + base + item) : -1);
         }
         uint4 cw[4];
         uint32_t sw[4];
 #pragma unroll
         for (int pass = 0; pass < 4; ++pass) {
+          const int item = pass * 16 + (tid >> 4);
           const bool valid = pos[pass] >= 0 && pos[pass] < nb;
           if (!valid && pos[pass] != -1) flag_error(dev_err, CSA2_DEVERR_INDEX_RANGE);
           const int64_t row = seq_row0 + (valid ? pos[pass] : 0);
-          cw[pass] = valid ? ldg_nc_v4(codes + row * (D / 2) + 16 * r) : make_uint4(0u, 0u, 0u, 0u);
-          sw[pass] = valid ? __ldg(reinterpret_cast<const uint16_t*>(scales + row * (D / 16)) + r) : 0u;
+          if (staged) {  // fetched during the previous tile (zeros where the position is invalid)
+            const uint8_t* rr = sm.raw + item * kRawRow;
+            cw[pass] = *reinterpret_cast<const uint4*>(rr + 16 * r);
+            sw[pass] = *reinterpret_cast<const uint16_t*>(rr + D / 2 + 2 * r);
+          } else {
+            cw[pass] = valid ? ldg_nc_v4(codes + row * (D / 2) + 16 * r) : make_uint4(0u, 0u, 0u, 0u);
+            sw[pass] = valid ? __ldg(reinterpret_cast<const uint16_t*>(scales + row * (D / 16)) + r) : 0u;
+          }
         }
 #pragma unroll
         for (int pass = 0; pass < 4; ++pass) {
@@ -240,9 +279,11 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int slot = base + item;
           const bool valid = item < count && slot < sl;
           const int64_t srow = static_cast<int64_t>(sb) * S + slo + (valid ? slot : 0);
-          const uint8_t* rowp = swa + srow * D + 32 * r;
+          // thread r takes channels 16r .. 16r + 15 and 256 + 16r .. + 15: each load of the 16
+          // threads of an item is 256 contiguous bytes
+          const uint8_t* rowp = swa + srow * D + 16 * r;
           e[pass][0] = valid ? ldg_nc_v4(rowp) : make_uint4(0u, 0u, 0u, 0u);
-          e[pass][1] = valid ? ldg_nc_v4(rowp + 16) : make_uint4(0u, 0u, 0u, 0u);
+          e[pass][1] = valid ? ldg_nc_v4(rowp + D / 2) : make_uint4(0u, 0u, 0u, 0u);
           iscale[pass] = valid ? __ldg(swa_scale + srow) : 1.0f;
         }
 #pragma unroll
@@ -258,8 +299,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             hv[2 * k + 1] = e4m3x2_to_h2(ew[k] >> 16);
           }
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<uint4*>(vrow + swz1024(item, 4 * r + k)) =
+          for (int k = 0; k < 4; ++k)  // chunks 2r, 2r + 1, 32 + 2r, 33 + 2r
+            *reinterpret_cast<uint4*>(vrow + swz1024(item, 2 * r + (k & 1) + 32 * (k >> 1))) =
                 make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
           if (r == 0) {
             sm.item_valid[item] = valid;
@@ -269,6 +310,22 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     __syncthreads();
+    // every read of sm.raw for this tile is done: request the next MXFP4 tile's rows
+    if (next_mx) {
+      const int r = tid & 15;
+#pragma unroll
+      for (int pass = 0; pass < 4; ++pass) {
+        const int item = pass * 16 + (tid >> 4);
+        const bool valid = pos_next[pass] >= 0 && pos_next[pass] < nb;
+        const int64_t row = seq_row0 + (valid ? pos_next[pass] : 0);
+        uint8_t* rr = sm.raw + item * kRawRow;
+        cp_async16(rr + 16 * r, codes + row * (D / 2) + 16 * r, valid ? 16u : 0u);
+        if (r < 2) cp_async16(rr + D / 2 + 16 * r, scales + row * (D / 16) + 16 * r, valid ? 16u : 0u);
+        pos_staged[pass] = pos_next[pass];
+      }
+      cp_async_commit();
+    }
+    staged = next_mx;
     if (warp == 0) {
       // P scale for SWA tiles: brings the largest token scale to [1, 2)
       float smax = 0.0f;
@@ -301,14 +358,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       float* zp = sm.zp[kh];
       const int i0 = 16 * ig + 2 * c;
-      zp[g * kTile + i0] = acc0[0];
-      zp[g * kTile + i0 + 1] = acc0[1];
-      zp[(g + 8) * kTile + i0] = acc0[2];
-      zp[(g + 8) * kTile + i0 + 1] = acc0[3];
-      zp[g * kTile + i0 + 8] = acc1[0];
-      zp[g * kTile + i0 + 9] = acc1[1];
-      zp[(g + 8) * kTile + i0 + 8] = acc1[2];
-      zp[(g + 8) * kTile + i0 + 9] = acc1[3];
+      *reinterpret_cast<float2*>(zp + g * kZs + i0) = make_float2(acc0[0], acc0[1]);
+      *reinterpret_cast<float2*>(zp + (g + 8) * kZs + i0) = make_float2(acc0[2], acc0[3]);
+      *reinterpret_cast<float2*>(zp + g * kZs + i0 + 8) = make_float2(acc1[0], acc1[1]);
+      *reinterpret_cast<float2*>(zp + (g + 8) * kZs + i0 + 8) = make_float2(acc1[2], acc1[3]);
     }
     __syncthreads();
 
@@ -320,10 +373,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int h = 2 * warp + hh;
         const float uh = sm.q_unscale[h];
         const float z0 = sm.item_valid[lane]
-                             ? (sm.zp[0][h * kTile + lane] + sm.zp[1][h * kTile + lane]) * uh * sm.item_scale[lane]
+                             ? (sm.zp[0][h * kZs + lane] + sm.zp[1][h * kZs + lane]) * uh * sm.item_scale[lane]
                              : -INFINITY;
         const float z1 = sm.item_valid[lane + 32]
-                             ? (sm.zp[0][h * kTile + lane + 32] + sm.zp[1][h * kTile + lane + 32]) * uh *
+                             ? (sm.zp[0][h * kZs + lane + 32] + sm.zp[1][h * kZs + lane + 32]) * uh *
                                    sm.item_scale[lane + 32]
                              : -INFINITY;
         float mt = fmaxf(z0, z1);
@@ -391,6 +444,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
     }
+    if (staged) cp_async_wait_all();  // the next tile's rows have landed (made visible below)
     __syncthreads();
   }
 
@@ -536,7 +590,7 @@ cudaError_t launch_attend(const void* q, float softmax_scale, const uint8_t* cod
     configured_device = dev;
   }
   profile_begin(CSA2_KERNEL_ATTEND, s);
-  cudaError_t e = launch_pdl(attend_kernel, dim3(splits, B), dim3(kThreads), smem, s,
+  cudaError_t e = launch_pdl(attend_kernel, dim3(B, splits), dim3(kThreads), smem, s,
                              static_cast<const uint16_t*>(q), softmax_scale, codes, scales, n_cap,
                              N, idx, K, swa, swa_scale, swa_len, W, qseq, swa_lo, S, nseq, out,
                              lse, part_o, part_ml,

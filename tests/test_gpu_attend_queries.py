@@ -120,3 +120,22 @@ def test_bad_sequences_and_windows_are_flagged(gpu):
     check_attention(out[0], lse[0], ro, rl)
     ro, rl = _oracle_query(q[2], codes, scales, 1, idx[2], swa, swsc, 60, 4)
     check_attention(out[2], lse[2], ro, rl)
+
+
+def test_more_queries_than_one_grid_dimension_row(gpu):
+    """70,000 queries: more than the 65,535 blocks a grid's y or z dimension can hold."""
+    B, n_cap, K = 1, 1024, 64
+    N = [1024]
+    cache, codes, scales, _, _ = build_cache(B, n_cap, N, 0, [0], seed=12, dev=gpu)
+    Q = 70000
+    rng = np.random.default_rng(12)
+    base = np.stack([np.sort(rng.choice(1024, K, replace=False)) for _ in range(16)]).astype(np.int32)
+    idx = base[np.arange(Q) % 16]
+    g = torch.Generator().manual_seed(13)
+    q = (torch.randn(16, 16, 512, generator=g) / math.sqrt(512)).to(torch.bfloat16)
+    qq = q[torch.arange(Q) % 16]
+    out, lse, err = _run_queries(qq, cache, N, [0] * Q, idx, None, None, None, None, 0, gpu)
+    assert err == 0
+    for i in (0, 1, 65534, 65535, 65536, Q - 1):
+        ro, rl = _oracle_query(q[i % 16], codes, scales, 0, idx[i], None, None, 0, 0)
+        check_attention(out[i], lse[i], ro, rl)
