@@ -100,6 +100,22 @@ def scan_traffic_per_launch(wl):
         return None
 
 
+def ced_traffic_per_launch(tokens):
+    """DRAM bytes per CED launch from the committed ncu capture (profiles/ced_quant_traffic.json),
+    scaled by token rows; None once the kernel's sources differ from the captured ones."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "ced_quant_traffic.json")) as f:
+            cap = json.load(f)
+        csrc = os.path.join(ROOT, "sparse_attention_decode_kv_b200", "csrc")
+        text = "".join(open(os.path.join(csrc, n)).read() for n in ("ced.cu", "tcgen05.cuh", "common.cuh"))
+        if hashlib.sha256(text.encode()).hexdigest() != cap["source_sha256"]:
+            return None
+        return int(round(cap["dram_bytes_per_token"] * tokens))
+    except Exception:
+        return None
+
+
 def algorithmic_bytes(wl) -> dict:
     """Bytes the step must move (indexer keys + gathered MXFP4 entries + scales + SWA rows)."""
     full = wl.B * wl.N * 128
@@ -729,7 +745,9 @@ def run_ced(args, world, rank, local):
                      "bound": "tensor", "achieved": round(tflops, 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "peak_kind": peak_kind,
                      "algorithmic_flop_per_launch": flop, "launch_ms": round(ms, 4),
-                     "traffic": None},
+                     "traffic": ced_traffic_per_launch(B * n),
+                     "algorithmic_bytes_per_launch": h.numel() * 2 + w.numel() * 2
+                     + codes.numel() + scales.numel()},
         "gpu_launches": per_step_launches * K,
         "clocks": clocks.summary(),
     }
