@@ -52,6 +52,10 @@ def _declare(L):
     L.oracle_ced_project.argtypes = [_P, _P, ctypes.c_int64, ctypes.c_int, _P, _P]
     L.oracle_mxfp4_dequantize_entry.argtypes = [_P, _P, _P]
     L.oracle_swa_quantize_token.argtypes = [_P, _P, _P]
+    L.oracle_f64_to_bf16.restype = ctypes.c_uint16
+    L.oracle_f64_to_bf16.argtypes = [ctypes.c_double]
+    L.oracle_swa_replay.argtypes = [_P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P,
+                                    ctypes.c_int]
     L.oracle_append.restype = ctypes.c_int
     L.oracle_append.argtypes = [_P, _P, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P, _P, _P,
                                 _P, _P, ctypes.c_int]
@@ -140,6 +144,28 @@ def ced_project(h_bits, w_bits):
     a = np.zeros((M, 512), np.float64)
     lib().oracle_ced_project(_ptr(h), _ptr(w), M, d, _ptr(c), _ptr(a))
     return c, a
+
+
+def f64_to_bf16(x) -> np.ndarray:
+    """float64 values -> bf16 bit patterns (uint16), one rounding to nearest even."""
+    xs = np.asarray(x, np.float64)
+    L = lib()
+    return np.array([L.oracle_f64_to_bf16(float(v)) for v in xs.ravel()], np.uint16).reshape(xs.shape)
+
+
+def swa_replay(h_bits, w_bits, N, swa, swa_scale):
+    """SWA bounded replay [A abstract; Juju Radar note; T1 "最后的结果"]: rebuild ring slots from
+    the last Wr tokens' hidden states. h_bits uint16 [B, Wr, d]; w_bits uint16 [512, d]; N [B];
+    swa uint8 [B, W, 512] and swa_scale float32 [B, W] are updated in place (other slots kept)."""
+    h = _c(h_bits, np.uint16)
+    w = _c(w_bits, np.uint16)
+    B, Wr, d = h.shape
+    assert w.shape == (512, d)
+    n = _c(N, np.int32)
+    assert swa.dtype == np.uint8 and swa.flags.c_contiguous and swa.shape[0] == B
+    assert swa_scale.dtype == np.float32 and swa_scale.flags.c_contiguous
+    W = swa.shape[1]
+    lib().oracle_swa_replay(_ptr(h), _ptr(w), B, Wr, d, _ptr(n), _ptr(swa), _ptr(swa_scale), W)
 
 
 def mxfp4_dequantize(codes, scales) -> np.ndarray:

@@ -353,6 +353,79 @@ void oracle_ced_project(const uint16_t *h, const uint16_t *w, int64_t M, int d, 
 }
 
 /* ------------------------------------------------------------------------------------------ */
+/* Rounding of a double to bf16, nearest-even, by its definition: with |x| = m 2^e, m in       */
+/* [0.5, 1), a normal bf16 keeps 8 significant bits (fewer below 2^-126, where the spacing     */
+/* stays 2^-133); the scaled significand is rounded to an integer with ties to even, once.     */
+/* Values above the largest finite bf16 after rounding become infinities.                      */
+/* ------------------------------------------------------------------------------------------ */
+uint16_t oracle_f64_to_bf16(double x) {
+  const int neg = signbit(x) != 0;
+  double a = fabs(x);
+  uint16_t out;
+  if (isnan(x)) return 0x7FC0;
+  if (a == 0.0 || isinf(a)) {
+    out = a == 0.0 ? 0x0000 : 0x7F80;
+  } else {
+    int e;
+    double m = frexp(a, &e);                   /* a = m * 2^e, m in [0.5, 1) */
+    int bits = 8;                              /* significant bits kept */
+    if (e - 1 < -126) bits -= (-126 - (e - 1)); /* bf16 subnormal: spacing 2^-133 */
+    double r;
+    if (bits < 0) {
+      r = 0.0;                                 /* below half the smallest subnormal */
+    } else {
+      double q = ldexp(m, bits);               /* exact */
+      double f = floor(q), d = q - f;
+      r = f;
+      if (d > 0.5 || (d == 0.5 && fmod(f, 2.0) != 0.0)) r = f + 1.0;
+    }
+    double v = ldexp(r, e - bits);             /* the rounded value, exact in double */
+    if (v > 3.3895313892515355e38) {           /* (2 - 2^-7) * 2^127 */
+      out = 0x7F80;
+    } else {
+      float fv = (float)v;                     /* exact: v has at most 8 significant bits */
+      uint32_t u;
+      memcpy(&u, &fv, sizeof u);
+      out = (uint16_t)(u >> 16);
+    }
+  }
+  return (uint16_t)(out | (neg ? 0x8000 : 0));
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* SWA bounded replay [A: "SWA Bounded Replay" keeps the persistent (host / SSD) KV cache at   */
+/* about 1/8 of DeepSeek-V4-Flash's; Juju Radar's note on the report: the persistent cache      */
+/* rebuilds the local sliding-window state instead of storing it; T1 "最后的结果": persistent   */
+/* KV cache (SSD / host memory) about 1/8].                                                     */
+/* Reading: the persisted copy of a sequence holds its global KV (MXFP4 codes and scales) and   */
+/* its indexer keys; a restore copies those rows back and rebuilds the FP8 SWA ring from the    */
+/* hidden states of the last Wr tokens: token r of sequence b sits at position                 */
+/* p = N[b] - Wr + r (rows with p < 0 do not exist and are skipped); its SWA row is             */
+/* x[j] = bf16_RNE(sum_k h[k] w[j][k]) (w holds one row per SWA channel; the sum is exact up to */
+/* double rounding), quantised with the SWA codec into ring slot p mod W -- the row an append   */
+/* of x at position p writes. Slots of other positions are left as they are.                   */
+/* ------------------------------------------------------------------------------------------ */
+void oracle_swa_replay(const uint16_t *h, const uint16_t *w, int B, int Wr, int d,
+                       const int32_t *N, uint8_t *swa_e4m3, float *swa_scale, int W) {
+  uint16_t x[CSA2O_D];
+  for (int b = 0; b < B; ++b) {
+    for (int r = 0; r < Wr; ++r) {
+      int64_t p = (int64_t)N[b] - Wr + r;
+      if (p < 0) continue;
+      const uint16_t *hr = h + ((int64_t)b * Wr + r) * d;
+      for (int j = 0; j < CSA2O_D; ++j) {
+        const uint16_t *wr = w + (int64_t)j * d;
+        double acc = 0.0;
+        for (int k = 0; k < d; ++k) acc += (double)bf16_to_f32(hr[k]) * (double)bf16_to_f32(wr[k]);
+        x[j] = oracle_f64_to_bf16(acc);
+      }
+      int64_t slot = (int64_t)b * W + (p % W);
+      oracle_swa_quantize_token(x, swa_e4m3 + slot * CSA2O_D, swa_scale + slot);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------------------------ */
 /* Full-mode indexer for one sequence [T1 hierarchical sparse indexer]:                        */
 /*   scores over all N entries; Top-K positions; block maxima over 8-position blocks;          */
 /*   Top-P blocks; pool = the selected blocks' positions in ascending block order, -1 past N.  */

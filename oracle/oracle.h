@@ -25,6 +25,9 @@ void oracle_ced_project(const uint16_t *h, const uint16_t *w, int64_t M, int d, 
 void oracle_mxfp4_quantize_entry(const uint16_t *x, uint8_t *codes, uint8_t *scales);
 void oracle_mxfp4_dequantize_entry(const uint8_t *codes, const uint8_t *scales, double *out);
 void oracle_swa_quantize_token(const uint16_t *x, uint8_t *e, float *scale);
+uint16_t oracle_f64_to_bf16(double x);
+void oracle_swa_replay(const uint16_t *h, const uint16_t *w, int B, int Wr, int d,
+                       const int32_t *N, uint8_t *swa_e4m3, float *swa_scale, int W);
 int oracle_append(const uint16_t *x, const uint16_t *ik, int B, int n, const int32_t *pos,
                   int n_cap, uint8_t *codes, uint8_t *scales, uint16_t *ik_cache,
                   uint8_t *swa_e4m3, float *swa_scale, int W);

@@ -37,6 +37,16 @@ MUTANTS = {
                                  "return (uint8_t)(mag | (r < 0 ? 8 : 0));"),
     "ring slot off by one": ("int64_t slot = (int64_t)b * W + (p % W);",
                              "int64_t slot = (int64_t)b * W + ((p + 1) % W);"),
+    "bf16 rounding ties away from zero": (
+        "if (d > 0.5 || (d == 0.5 && fmod(f, 2.0) != 0.0)) r = f + 1.0;",
+        "if (d >= 0.5) r = f + 1.0;"),
+    "replay window starts one token late": ("int64_t p = (int64_t)N[b] - Wr + r;",
+                                            "int64_t p = (int64_t)N[b] - Wr + r + 1;"),
+    "replay reads the projection transposed": (
+        "acc += (double)bf16_to_f32(hr[k]) * (double)bf16_to_f32(wr[k]);",
+        "acc += (double)bf16_to_f32(hr[k]) * (double)bf16_to_f32(w[(int64_t)k * CSA2O_D + j]);"),
+    "projection drops the last term": ("      for (int k = 0; k < d; ++k) {\n        double p =",
+                                       "      for (int k = 0; k < d - 1; ++k) {\n        double p ="),
     "query/key operands swapped": (
         "dot += (double)bf16_to_f32(iq[h * CSA2O_DI + i]) * (double)bf16_to_f32(k[i]);",
         "dot += (double)bf16_to_f32(iq[i]) * (double)bf16_to_f32(k[h * 0 + i]);"),
@@ -56,7 +66,8 @@ def _run(name):
         with open(os.path.join(d, "oracle", "oracle.c"), "w") as f:
             f.write(src.replace(old, new))
         r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                            "tests/test_oracle_codecs.py", "tests/test_oracle_index_attend.py"],
+                            "tests/test_oracle_codecs.py", "tests/test_oracle_index_attend.py",
+                            "tests/test_oracle_ced.py", "tests/test_oracle_replay.py"],
                            cwd=d, capture_output=True, text=True, timeout=600)
         return name, r.returncode
     finally:
