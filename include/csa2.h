@@ -130,6 +130,62 @@ CSA2_API int csa2_ced_project_quant(const void *h, const void *w, int B, int n, 
                                     uint8_t *scales, int32_t *dev_err, csa2_stream_t stream);
 
 /*
+ * SWA bounded replay, part 1: restore a persisted sequence's cache rows from host memory.
+ * Defines: "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache Compression", abstract (SWA
+ * Bounded Replay brings the persistent KV cache on SSD or in host memory to about 1/8 of
+ * DeepSeek-V4-Flash's), and the Juju Radar note on that report (the persistent cache rebuilds
+ * the local sliding-window state instead of storing it). Reading: what persists is the global KV
+ * (MXFP4 codes and scales) and the indexer keys; the FP8 SWA ring is rebuilt by
+ * csa2_swa_replay.
+ *   host_codes   uint8 [B, n_host, 256], host_scales uint8 [B, n_host, 32], host_ik bf16
+ *                [B, n_host, 64] or NULL: the persisted rows (host memory; page-locked memory
+ *                lets the copies run asynchronously on the stream, pageable memory makes the
+ *                call return only after them).
+ *   N            HOST int32 [B]: rows 0 .. N[b]-1 of sequence b are copied; 0 <= N[b] <=
+ *                min(n_host, n_cap).
+ *   codes, scales, ik_cache: the device cache (as csa2_append_quant); ik_cache NULL exactly when
+ *                host_ik is NULL. Rows N[b] .. n_cap-1 are not touched.
+ * Copies only (cudaMemcpyAsync on the stream; runs of full sequences are merged into one copy);
+ * launches no kernel. Errors: CSA2_ERR_INVALID for bad sizes or pointers, CSA2_ERR_CUDA when a
+ * copy cannot be queued.
+ */
+CSA2_API int csa2_cache_restore(const uint8_t *host_codes, const uint8_t *host_scales,
+                                const void *host_ik, int B, int n_host, const int32_t *N,
+                                int n_cap, uint8_t *codes, uint8_t *scales, void *ik_cache,
+                                csa2_stream_t stream);
+
+/*
+ * The inverse copy: rows 0 .. N[b]-1 of the device cache to the host layout above (the state a
+ * later csa2_cache_restore reads). Same arguments, same rules, directions swapped.
+ */
+CSA2_API int csa2_cache_persist(const uint8_t *codes, const uint8_t *scales, const void *ik_cache,
+                                int B, int n_cap, const int32_t *N, int n_host,
+                                uint8_t *host_codes, uint8_t *host_scales, void *host_ik,
+                                csa2_stream_t stream);
+
+/*
+ * SWA bounded replay, part 2: rebuild the FP8 SWA ring of B restored sequences from the hidden
+ * states of their last Wr tokens (same sources as csa2_cache_restore). Token r of sequence b is
+ * position p = N[b] - Wr + r; its SWA row is x = bf16_RNE(h w^T) (bf16 inputs, fp32 accumulation
+ * on the tcgen05 tensor cores), quantised with csa2_append_quant's SWA codec into ring slot
+ * p mod W, so the slot holds exactly what an append of x at position p would have written.
+ * Positions p < 0 (a sequence shorter than the window) are skipped; other slots are not touched.
+ *   h         bf16 [B, Wr, d]: hidden states of the window tokens, oldest first.
+ *   w         bf16 [512, d]: the layer's SWA KV projection, one row per channel.
+ *   d         a multiple of CSA2_CED_D_ALIGN (64), at most CSA2_MAX_CED_D.
+ *   N         device int32 [B]: tokens in each sequence (a negative N[b] skips the sequence and
+ *             flags CSA2_DEVERR_NLEN).
+ *   swa, swa_scale, W: the ring (as csa2_append_quant); 1 <= Wr <= W.
+ *   ws        device workspace of csa2_swa_replay_workspace_bytes(B, Wr, d) bytes (fp32 partial
+ *             sums of the split reduction), 16-byte aligned.
+ * Launches two kernels (the split-K projection and the sum-round-quantise pass).
+ */
+CSA2_API size_t csa2_swa_replay_workspace_bytes(int B, int Wr, int d);
+CSA2_API int csa2_swa_replay(const void *h, const void *w, int B, int Wr, int d, const int32_t *N,
+                             uint8_t *swa, float *swa_scale, int W, void *ws, size_t ws_bytes,
+                             int32_t *dev_err, csa2_stream_t stream);
+
+/*
  * Full-mode indexer: scores every entry, selects the Top-K positions, takes block maxima over
  * 8-position blocks, selects the Top-P blocks and writes the pool.
  * Defines: the hierarchical sparse indexer paragraph of section 一 (Top-512, 2048 blocks x 8).
@@ -239,7 +295,8 @@ enum {
   CSA2_KERNEL_REINDEX = 3,     /* Reindex score + select (two kernels) */
   CSA2_KERNEL_ATTEND = 4,      /* attention + merge (one or two kernels) */
   CSA2_KERNEL_CED = 5,         /* CED projection with the MXFP4 epilogue */
-  CSA2_KERNEL_COUNT = 6
+  CSA2_KERNEL_REPLAY = 6,      /* SWA replay: projection + sum/round/quantise (two kernels) */
+  CSA2_KERNEL_COUNT = 7
 };
 CSA2_API int csa2_set_profile_events(int kernel, void *start_event, void *stop_event);
 

@@ -57,6 +57,11 @@ def lib() -> ctypes.CDLL:
                                   Z, P, P]
         L.csa2_attend_queries.argtypes = [P, ctypes.c_float, P, P, I, I, P, P, P, I, P, P, I, P, P,
                                           I, I, P, P, P, Z, P, P]
+        L.csa2_cache_restore.argtypes = [P, P, P, I, I, P, I, P, P, P, P]
+        L.csa2_cache_persist.argtypes = [P, P, P, I, I, P, I, P, P, P, P]
+        L.csa2_swa_replay_workspace_bytes.argtypes = [I, I, I]
+        L.csa2_swa_replay_workspace_bytes.restype = Z
+        L.csa2_swa_replay.argtypes = [P, P, I, I, I, P, P, P, I, P, Z, P, P]
         L.csa2_status_string.argtypes = [I]
         L.csa2_status_string.restype = ctypes.c_char_p
         L.csa2_launch_count.restype = ctypes.c_uint64
@@ -89,6 +94,26 @@ def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor"):
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _hptr(t: Optional[torch.Tensor], dtype, name="tensor"):
+    """Pointer of a host (CPU) tensor; page-locked memory lets the copies run asynchronously."""
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_counts(N, B):
+    vals = [int(v) for v in N]
+    if len(vals) != B:
+        raise ValueError(f"N must hold {B} counts")
+    return (ctypes.c_int32 * B)(*vals)
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -131,6 +156,56 @@ def ced_project_quant(h, w, pos, codes, scales, dev_err=None, stream=None) -> No
         _ptr(scales, torch.uint8, "scales"), _ptr(dev_err, torch.int32, "dev_err"),
         _stream(stream))
     _check("csa2_ced_project_quant", st)
+
+
+def cache_restore(host_codes, host_scales, host_ik, N, codes, scales, ik_cache=None,
+                  stream=None) -> None:
+    """SWA bounded replay, restore side: copy rows 0 .. N[b]-1 of the persisted MXFP4 cache (and
+    indexer keys) from host tensors [B, n_host, ...] into the device cache [B, n_cap, ...].
+    N is a host sequence of B ints."""
+    B, n_host = host_codes.shape[0], host_codes.shape[1]
+    n_cap = codes.shape[1]
+    n = _host_counts(N, B)
+    st = lib().csa2_cache_restore(
+        _hptr(host_codes, torch.uint8, "host_codes"), _hptr(host_scales, torch.uint8, "host_scales"),
+        _hptr(host_ik, torch.bfloat16, "host_ik"), B, n_host, n, n_cap,
+        _ptr(codes, torch.uint8, "codes"), _ptr(scales, torch.uint8, "scales"),
+        _ptr(ik_cache, torch.bfloat16, "ik_cache"), _stream(stream))
+    _check("csa2_cache_restore", st)
+
+
+def cache_persist(codes, scales, ik_cache, N, host_codes, host_scales, host_ik=None,
+                  stream=None) -> None:
+    """The inverse of cache_restore: rows 0 .. N[b]-1 of the device cache to host tensors."""
+    B, n_cap = codes.shape[0], codes.shape[1]
+    n_host = host_codes.shape[1]
+    n = _host_counts(N, B)
+    st = lib().csa2_cache_persist(
+        _ptr(codes, torch.uint8, "codes"), _ptr(scales, torch.uint8, "scales"),
+        _ptr(ik_cache, torch.bfloat16, "ik_cache"), B, n_cap, n, n_host,
+        _hptr(host_codes, torch.uint8, "host_codes"), _hptr(host_scales, torch.uint8, "host_scales"),
+        _hptr(host_ik, torch.bfloat16, "host_ik"), _stream(stream))
+    _check("csa2_cache_persist", st)
+
+
+def swa_replay_workspace_bytes(B: int, Wr: int, d: int) -> int:
+    return int(lib().csa2_swa_replay_workspace_bytes(B, Wr, d))
+
+
+def swa_replay(h, w, N, swa, swa_scale, ws, dev_err=None, stream=None) -> None:
+    """SWA bounded replay: ring slot (N[b] - Wr + r) mod W of sequence b gets the SWA codec of
+    bf16_RNE(h[b, r] w^T). h bf16 [B, Wr, d]; w bf16 [512, d]; N int32 [B] (device);
+    swa uint8 [B, W, 512]; swa_scale f32 [B, W]; ws of swa_replay_workspace_bytes bytes."""
+    B, Wr, d = h.shape
+    if tuple(w.shape) != (D, d):
+        raise ValueError(f"w must be [{D}, {d}], got {tuple(w.shape)}")
+    W = swa.shape[1]
+    st = lib().csa2_swa_replay(
+        _ptr(h, torch.bfloat16, "h"), _ptr(w, torch.bfloat16, "w"), B, Wr, d,
+        _ptr(N, torch.int32, "N"), _ptr(swa, torch.uint8, "swa"),
+        _ptr(swa_scale, torch.float32, "swa_scale"), W, _ptr(ws, None, "ws"),
+        ws.numel() * ws.element_size(), _ptr(dev_err, torch.int32, "dev_err"), _stream(stream))
+    _check("csa2_swa_replay", st)
 
 
 def index_full_workspace_bytes(B: int, n_cap: int, K: int, P: int) -> int:

@@ -69,11 +69,48 @@ bool ptr_ok(const void* p, bool nullable = false) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA; }
 
+// Rows 0 .. N[b]-1 of every sequence between two [B, rows, row_bytes] layouts. A run of
+// sequences that are full in both layouts is contiguous, so it goes as one copy.
+cudaError_t copy_rows(void* dst, int64_t dst_rows, const void* src, int64_t src_rows,
+                      int64_t row_bytes, int B, const int32_t* N, cudaMemcpyKind kind,
+                      cudaStream_t s) {
+  int b = 0;
+  while (b < B) {
+    int e = b + 1;
+    int64_t rows = N[b];
+    while (e < B && N[e - 1] == dst_rows && N[e - 1] == src_rows) rows += N[e++];
+    if (rows > 0) {
+      cudaError_t err = cudaMemcpyAsync(
+          static_cast<uint8_t*>(dst) + static_cast<int64_t>(b) * dst_rows * row_bytes,
+          static_cast<const uint8_t*>(src) + static_cast<int64_t>(b) * src_rows * row_bytes,
+          static_cast<size_t>(rows * row_bytes), kind, s);
+      if (err != cudaSuccess) return err;
+    }
+    b = e;
+  }
+  return cudaSuccess;
+}
+
+// The checks shared by csa2_cache_restore and csa2_cache_persist.
+int cache_copy_args_ok(const void* codes, const void* scales, const void* ik, int B, int n_cap,
+                       const int32_t* N, int n_host, const void* h_codes, const void* h_scales,
+                       const void* h_ik) {
+  if (B <= 0 || n_cap <= 0 || (n_cap % CSA2_S) != 0 || n_host < 0) return CSA2_ERR_INVALID;
+  if (B > CSA2_MAX_B || n_cap > CSA2_MAX_NCAP || n_host > CSA2_MAX_NCAP) return CSA2_ERR_UNSUPPORTED;
+  if (N == nullptr || !ptr_ok(codes) || !ptr_ok(scales) || !ptr_ok(h_codes) || !ptr_ok(h_scales))
+    return CSA2_ERR_INVALID;
+  if ((ik == nullptr) != (h_ik == nullptr) || !ptr_ok(ik, true) || !ptr_ok(h_ik, true))
+    return CSA2_ERR_INVALID;
+  for (int b = 0; b < B; ++b)
+    if (N[b] < 0 || N[b] > n_cap || N[b] > n_host) return CSA2_ERR_INVALID;
+  return CSA2_OK;
+}
+
 }  // namespace
 
 extern "C" {
 
-int csa2_abi_version(void) { return 2; }
+int csa2_abi_version(void) { return 3; }
 
 uint64_t csa2_launch_count(void) { return csa2::g_launches.load(); }
 
@@ -230,6 +267,59 @@ int csa2_attend_queries(const void* q, float softmax_scale, const uint8_t* codes
                                          W > 0 ? swa_len : nullptr, W, qseq,
                                          W > 0 ? swa_lo : nullptr, S, B, Q, out, lse, ws, dev_err,
                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int csa2_cache_restore(const uint8_t* host_codes, const uint8_t* host_scales, const void* host_ik,
+                       int B, int n_host, const int32_t* N, int n_cap, uint8_t* codes,
+                       uint8_t* scales, void* ik_cache, csa2_stream_t stream) {
+  const int st = cache_copy_args_ok(codes, scales, ik_cache, B, n_cap, N, n_host, host_codes,
+                                    host_scales, host_ik);
+  if (st != CSA2_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = copy_rows(codes, n_cap, host_codes, n_host, CSA2_D / 2, B, N,
+                            cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = copy_rows(scales, n_cap, host_scales, n_host, CSA2_D / 16, B, N, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && ik_cache != nullptr)
+    e = copy_rows(ik_cache, n_cap, host_ik, n_host, CSA2_DI * 2, B, N, cudaMemcpyHostToDevice, s);
+  return cuda_status(e);
+}
+
+int csa2_cache_persist(const uint8_t* codes, const uint8_t* scales, const void* ik_cache, int B,
+                       int n_cap, const int32_t* N, int n_host, uint8_t* host_codes,
+                       uint8_t* host_scales, void* host_ik, csa2_stream_t stream) {
+  const int st = cache_copy_args_ok(codes, scales, ik_cache, B, n_cap, N, n_host, host_codes,
+                                    host_scales, host_ik);
+  if (st != CSA2_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = copy_rows(host_codes, n_host, codes, n_cap, CSA2_D / 2, B, N,
+                            cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess)
+    e = copy_rows(host_scales, n_host, scales, n_cap, CSA2_D / 16, B, N, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && ik_cache != nullptr)
+    e = copy_rows(host_ik, n_host, ik_cache, n_cap, CSA2_DI * 2, B, N, cudaMemcpyDeviceToHost, s);
+  return cuda_status(e);
+}
+
+size_t csa2_swa_replay_workspace_bytes(int B, int Wr, int d) {
+  if (B <= 0 || Wr <= 0 || d < CSA2_CED_D_ALIGN || (d % CSA2_CED_D_ALIGN) != 0) return 0;
+  return csa2::swa_replay_workspace_bytes(B, Wr, d);
+}
+
+int csa2_swa_replay(const void* h, const void* w, int B, int Wr, int d, const int32_t* N,
+                    uint8_t* swa, float* swa_scale, int W, void* ws, size_t ws_bytes,
+                    int32_t* dev_err, csa2_stream_t stream) {
+  if (B <= 0 || Wr < 0 || W <= 0 || Wr > W) return CSA2_ERR_INVALID;
+  if (d < CSA2_CED_D_ALIGN || (d % CSA2_CED_D_ALIGN) != 0) return CSA2_ERR_INVALID;
+  if (B > CSA2_MAX_B || W > CSA2_MAX_W || d > CSA2_MAX_CED_D) return CSA2_ERR_UNSUPPORTED;
+  if (!ptr_ok(h) || !ptr_ok(w) || !ptr_ok(N) || !ptr_ok(swa) || !ptr_ok(swa_scale))
+    return CSA2_ERR_INVALID;
+  if (dev_err != nullptr && (reinterpret_cast<uintptr_t>(dev_err) & 3u)) return CSA2_ERR_INVALID;
+  if (Wr == 0) return CSA2_OK;
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < csa2::swa_replay_workspace_bytes(B, Wr, d))
+    return CSA2_ERR_WORKSPACE;
+  return cuda_status(csa2::launch_swa_replay(h, w, B, Wr, d, N, swa, swa_scale, W, ws, dev_err,
+                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

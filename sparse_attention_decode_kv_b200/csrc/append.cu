@@ -20,6 +20,7 @@
 // is then the E2M1 RNE of x/scale.
 #include "common.cuh"
 #include "internal.h"
+#include "swa_codec.cuh"
 
 namespace csa2 {
 
@@ -96,20 +97,8 @@ __global__ void __launch_bounds__(kAppendWarps * 32)
   // SWA ring: only the last W of the n new tokens survive, so only they are written (no two
   // writers of one slot within a call).
   if (swa != nullptr && W > 0 && i >= n - W) {
-    float amax = 0.0f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(v[k]));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-    const float s = __fdiv_rn(amax, 448.0f);
-    uint32_t e[4] = {0u, 0u, 0u, 0u};
-    if (s > 0.0f) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t two = cvt_e4m3x2(__fdiv_rn(v[2 * k], s), __fdiv_rn(v[2 * k + 1], s));
-        e[k >> 1] |= two << (16 * (k & 1));
-      }
-    }
+    uint32_t e[4];
+    const float s = swa_quantize_row_lane(v, e);
     const int64_t slot = static_cast<int64_t>(b) * W + (p % W);
     reinterpret_cast<uint4*>(swa + slot * D)[lane] = make_uint4(e[0], e[1], e[2], e[3]);
     if (lane == 0) swa_scale[slot] = s;

@@ -27,12 +27,26 @@
 //                       accumulator; meanwhile the MMAs of the next tile fill the other one.
 // Every mbarrier wait is bounded; a timeout flags CSA2_DEVERR_TIMEOUT, the producer drains its
 // own bulk copies, the MMA issuer still commits, and the tensor memory is always freed.
+//
+// SWA bounded replay. "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache Compression",
+// abstract: SWA Bounded Replay keeps the persistent (host / SSD) KV cache at about 1/8 of
+// DeepSeek-V4-Flash's; the Juju Radar note on the report: the persistent cache rebuilds the local
+// sliding-window state instead of storing it. Reading: a restored sequence gets its FP8 SWA ring
+// back from the hidden states of its last Wr tokens: token r of sequence b is position
+// p = N[b] - Wr + r, its SWA row is x = bf16_RNE(h w^T) (fp32 accumulation), quantised with the
+// append path's SWA codec into ring slot p mod W. Two kernels:
+//   replay_proj_kernel  the same persistent tcgen05 GEMM with the d-slices split over ksplit tile
+//                       groups (the window is a few hundred rows, so the K split is what fills the
+//                       SMs); the epilogue stores each fp32 partial accumulator row to a workspace.
+//   replay_swa_kernel   one warp per token row: adds the ksplit partials in a fixed order, rounds
+//                       to bf16, and applies the SWA codec (swa_codec.cuh) into the ring slot.
 #include <algorithm>
 #include <mutex>
 #include <vector>
 
 #include "common.cuh"
 #include "internal.h"
+#include "swa_codec.cuh"
 #include "tcgen05.cuh"
 
 namespace csa2 {
@@ -97,15 +111,51 @@ __device__ __forceinline__ uint2 quantize_group_f32(const float* v, uint32_t& sc
   return make_uint2(w[0], w[1]);
 }
 
-__global__ void __launch_bounds__(kCedThreads, 1)
-    ced_quant_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w,
-                     int M, int n, int d, const int32_t* __restrict__ pos, int n_cap,
-                     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int32_t* dev_err) {
+// What the epilogue does with a finished 128-row x 256-channel accumulator.
+enum ProjEpilogue : int {
+  kEpiMxfp4Cache = 0,  // quantise each 16-channel group into MXFP4 cache rows pos[b] + i
+  kEpiF32Partial = 1,  // store the fp32 partial sums of this tile's d-range to the workspace
+};
+
+struct ProjArgs {
+  int M;       // rows of h (tokens)
+  int n;       // rows per sequence (kEpiMxfp4Cache: token i of sequence b is row b n + i)
+  int d;       // reduction length, a multiple of kCedK
+  int ksplit;  // tile groups the d-slices are split over (1 for kEpiMxfp4Cache), <= d / kCedK
+  const int32_t* pos;
+  int n_cap;
+  uint8_t* codes;
+  uint8_t* scales;
+  float* part;  // kEpiF32Partial: [ksplit][M][512]
+  int32_t* dev_err;
+};
+
+// Tile t: channel half t % 2; then (t / 2) = token tile * ksplit + d-split.
+struct ProjTile {
+  int m0, n0, kb, ke, ks;
+};
+__device__ __forceinline__ ProjTile proj_tile(int t, int ksplit, int nk) {
+  ProjTile r;
+  r.n0 = (t & 1) * kCedN;
+  const int u = t >> 1;
+  const int mt = u / ksplit;
+  r.ks = u - mt * ksplit;
+  r.m0 = mt * kCedM;
+  r.kb = r.ks * nk / ksplit;
+  r.ke = (r.ks + 1) * nk / ksplit;
+  return r;
+}
+
+template <int kEpi>
+__device__ __forceinline__ void proj_body(const CUtensorMap* tm_h, const CUtensorMap* tm_w,
+                                          const ProjArgs& a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   CedSmem& sm = *reinterpret_cast<CedSmem*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nk = d / kCedK;
-  const int tiles = ((M + kCedM - 1) / kCedM) * (D / kCedN);
+  const int M = a.M, n = a.n, ksplit = a.ksplit;
+  const int nk = a.d / kCedK;
+  int32_t* dev_err = a.dev_err;
+  const int tiles = ((M + kCedM - 1) / kCedM) * (D / kCedN) * ksplit;
   const int my_tiles = tiles > static_cast<int>(blockIdx.x)
                            ? (tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
                            : 0;
@@ -140,8 +190,8 @@ __global__ void __launch_bounds__(kCedThreads, 1)
       int it = 0;  // stage uses so far (the ring runs on across tiles)
       for (int j = 0; j < my_tiles && !*abort; ++j) {
         const int t = static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x);
-        const int m0 = (t >> 1) * kCedM, n0 = (t & 1) * kCedN;
-        for (int kc = 0; kc < nk; ++kc, ++it) {
+        const ProjTile pt = proj_tile(t, ksplit, nk);
+        for (int kc = pt.kb; kc < pt.ke; ++kc, ++it) {
           const int s = it % kCedStages;
           if (it >= kCedStages &&
               !bounded_wait(&sm.empty[s], static_cast<uint32_t>(((it / kCedStages) & 1) ^ 1), abort)) {
@@ -150,8 +200,8 @@ __global__ void __launch_bounds__(kCedThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&sm.full[s], kCedATile + kCedBTile);
-          tma_load_2d(sm.a[s], &tm_h, &sm.full[s], kc * kCedK, m0);
-          tma_load_2d(sm.b[s], &tm_w, &sm.full[s], kc * kCedK, n0);
+          tma_load_2d(sm.a[s], tm_h, &sm.full[s], kc * kCedK, pt.m0);
+          tma_load_2d(sm.b[s], tm_w, &sm.full[s], kc * kCedK, pt.n0);
         }
       }
       // drain: every issued copy must land before the CTA may exit
@@ -173,8 +223,10 @@ __global__ void __launch_bounds__(kCedThreads, 1)
         }
         tcgen05_fence_after();
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kCedN);
+        const ProjTile pt = proj_tile(static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x),
+                                      ksplit, nk);
         bool ok = true;
-        for (int kc = 0; kc < nk; ++kc, ++it) {
+        for (int kc = pt.kb; kc < pt.ke; ++kc, ++it) {
           const int s = it % kCedStages;
           if (!bounded_wait(&sm.full[s], static_cast<uint32_t>((it / kCedStages) & 1), abort)) {
             if (!*abort) flag_error(dev_err, CSA2_DEVERR_TIMEOUT);
@@ -187,7 +239,7 @@ __global__ void __launch_bounds__(kCedThreads, 1)
 #pragma unroll
           for (int k4 = 0; k4 < kCedK / 16; ++k4)  // 16 bf16 = 32 bytes per instruction
             umma_bf16(d_tmem, umma_desc_k128(a0 + 32 * k4), umma_desc_k128(b0 + 32 * k4), kCedIdesc,
-                      (kc | k4) != 0 ? 1u : 0u);
+                      (kc != pt.kb || k4 != 0) ? 1u : 0u);
           umma_commit(&sm.empty[s]);  // the stage is free once these MMAs have read it
         }
         umma_commit(&sm.acc_full[acc]);  // every MMA issued so far has completed
@@ -200,7 +252,8 @@ __global__ void __launch_bounds__(kCedThreads, 1)
     for (int j = 0; j < my_tiles; ++j) {
       const int acc = j & 1;
       const int t = static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x);
-      const int m0 = (t >> 1) * kCedM, n0 = (t & 1) * kCedN;
+      const ProjTile pt = proj_tile(t, ksplit, nk);
+      const int m0 = pt.m0, n0 = pt.n0;
       const bool ok = __all_sync(0xFFFFFFFFu,
                                  bounded_wait(&sm.acc_full[acc], static_cast<uint32_t>((j >> 1) & 1), abort));
       if (!ok) {  // the MMA issuer gave up (and has flagged it) or the wait ran out
@@ -209,6 +262,32 @@ __global__ void __launch_bounds__(kCedThreads, 1)
       }
       tcgen05_fence_after();
       const int row = m0 + 32 * quarter + lane;
+      const uint32_t tbase =
+          tmem + static_cast<uint32_t>(acc * kCedN) + (static_cast<uint32_t>(32 * quarter) << 16);
+      if constexpr (kEpi == kEpiF32Partial) {
+        float* prow = a.part + (static_cast<int64_t>(pt.ks) * M + row) * D + n0;
+#pragma unroll 1
+        for (int g = 0; g < kCedN / 16; ++g) {
+          uint32_t r[16];
+          tmem_ld16(tbase + static_cast<uint32_t>(16 * g), r);
+          tmem_wait_ld();
+          if (row < M) {
+            float4* dst4 = reinterpret_cast<float4*>(prow + 16 * g);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst4[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                    __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+          }
+        }
+        tcgen05_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.acc_empty[acc]);
+        continue;
+      }
+      const int32_t* pos = a.pos;
+      const int n_cap = a.n_cap;
+      uint8_t* codes = a.codes;
+      uint8_t* scales = a.scales;
       int64_t dst = -1;
       if (row < M) {
         const int b = row / n, i = row - (row / n) * n;
@@ -216,8 +295,6 @@ __global__ void __launch_bounds__(kCedThreads, 1)
         if (p >= 0 && p < n_cap) dst = static_cast<int64_t>(b) * n_cap + p;
         else if (n0 == 0) flag_error(dev_err, CSA2_DEVERR_POS_RANGE);
       }
-      const uint32_t tbase =
-          tmem + static_cast<uint32_t>(acc * kCedN) + (static_cast<uint32_t>(32 * quarter) << 16);
       uint32_t sc[16];
 #pragma unroll 1
       for (int g = 0; g < kCedN / 16; ++g) {
@@ -262,57 +339,184 @@ __global__ void __launch_bounds__(kCedThreads, 1)
   }
 }
 
+__global__ void __launch_bounds__(kCedThreads, 1)
+    ced_quant_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w,
+                     const ProjArgs a) {
+  proj_body<kEpiMxfp4Cache>(&tm_h, &tm_w, a);
+}
+
+__global__ void __launch_bounds__(kCedThreads, 1)
+    replay_proj_kernel(const __grid_constant__ CUtensorMap tm_h,
+                       const __grid_constant__ CUtensorMap tm_w, const ProjArgs a) {
+  proj_body<kEpiF32Partial>(&tm_h, &tm_w, a);
+}
+
+// One warp per window row: sum of the partials (split 0 first), bf16 rounding, SWA codec.
+constexpr int kReplayWarps = 8;
+__global__ void __launch_bounds__(kReplayWarps * 32)
+    replay_swa_kernel(const float* __restrict__ part, int ksplit, int M, int Wr,
+                      const int32_t* __restrict__ N, uint8_t* __restrict__ swa,
+                      float* __restrict__ swa_scale, int W, int32_t* dev_err) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int row = static_cast<int>(blockIdx.x) * kReplayWarps + static_cast<int>(threadIdx.x >> 5);
+  if (row >= M) return;
+  const int b = row / Wr, r = row - (row / Wr) * Wr;
+  const int nb = __ldg(N + b);
+  if (nb < 0) {
+    if (lane == 0 && r == 0) flag_error(dev_err, CSA2_DEVERR_NLEN);
+    return;
+  }
+  const int64_t p = static_cast<int64_t>(nb) - Wr + r;
+  if (p < 0) return;  // the sequence is shorter than the window: no such token
+  float v[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = 0.0f;
+  for (int ks = 0; ks < ksplit; ++ks) {
+    const float4* src =
+        reinterpret_cast<const float4*>(part + (static_cast<int64_t>(ks) * M + row) * D + 16 * lane);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 f = __ldg(src + q);
+      v[4 * q] += f.x;
+      v[4 * q + 1] += f.y;
+      v[4 * q + 2] += f.z;
+      v[4 * q + 3] += f.w;
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __bfloat162float(__float2bfloat16_rn(v[k]));
+  uint32_t e[4];
+  const float s = swa_quantize_row_lane(v, e);
+  const int64_t slot = static_cast<int64_t>(b) * W + p % W;
+  reinterpret_cast<uint4*>(swa + slot * D)[lane] = make_uint4(e[0], e[1], e[2], e[3]);
+  if (lane == 0) swa_scale[slot] = s;
+}
+
 std::mutex g_ced_mu;
-std::vector<int> g_ced_ready;  // per device: shared-memory attribute set
+std::vector<int> g_ced_ready;  // per device: shared-memory attributes set
 
-}  // namespace
-
-cudaError_t launch_ced_quant(const void* h, const void* w, int B, int n, int d, const int32_t* pos,
-                             int n_cap, uint8_t* codes, uint8_t* scales, int32_t* dev_err,
-                             cudaStream_t s) {
+// Tensor maps of h [M, d] (boxes of 128 rows) and w [512, d] (boxes of 256 rows), 64-wide
+// d-slices with 128-byte swizzle.
+cudaError_t proj_tensor_maps(const void* h, const void* w, int64_t M, int d, CUtensorMap* map_h,
+                             CUtensorMap* map_w) {
   const TensorMapEncodeFn enc = tensor_map_encoder();
   if (enc == nullptr) return cudaErrorNotSupported;
-  const int64_t M = static_cast<int64_t>(B) * n;
-  CUtensorMap map_h, map_w;
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t estr[2] = {1, 1};
   {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(kCedK), static_cast<cuuint32_t>(kCedM)};
-    const cuuint32_t estr[2] = {1, 1};
-    if (enc(&map_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(h), dims, strides, box,
+    if (enc(map_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(h), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(D)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(kCedK), static_cast<cuuint32_t>(kCedN)};
-    const cuuint32_t estr[2] = {1, 1};
-    if (enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), dims, strides, box,
+    if (enc(map_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  return cudaSuccess;
+}
+
+cudaError_t proj_configure() {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  {
-    std::lock_guard<std::mutex> lock(g_ced_mu);
-    if (dev >= static_cast<int>(g_ced_ready.size())) g_ced_ready.resize(dev + 1, 0);
-    if (!g_ced_ready[dev]) {
-      e = cudaFuncSetAttribute(ced_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  std::lock_guard<std::mutex> lock(g_ced_mu);
+  if (dev >= static_cast<int>(g_ced_ready.size())) g_ced_ready.resize(dev + 1, 0);
+  if (!g_ced_ready[dev]) {
+    e = cudaFuncSetAttribute(ced_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sizeof(CedSmem)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(replay_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(sizeof(CedSmem)));
-      if (e != cudaSuccess) return e;
-      g_ced_ready[dev] = 1;
-    }
+    if (e != cudaSuccess) return e;
+    g_ced_ready[dev] = 1;
   }
+  return cudaSuccess;
+}
+
+constexpr int kReplayTargetCtas = 148;  // one B200's SMs: the K split aims to fill them once
+
+int replay_ksplit(int64_t M, int d) {
+  const int64_t mn_tiles = ((M + kCedM - 1) / kCedM) * (D / kCedN);
+  int64_t k = kReplayTargetCtas / std::max<int64_t>(mn_tiles, 1);
+  k = std::min<int64_t>(k, d / kCedK);
+  return static_cast<int>(std::max<int64_t>(k, 1));
+}
+
+}  // namespace
+
+cudaError_t launch_ced_quant(const void* h, const void* w, int B, int n, int d, const int32_t* pos,
+                             int n_cap, uint8_t* codes, uint8_t* scales, int32_t* dev_err,
+                             cudaStream_t s) {
+  const int64_t M = static_cast<int64_t>(B) * n;
+  CUtensorMap map_h, map_w;
+  cudaError_t e = proj_tensor_maps(h, w, M, d, &map_h, &map_w);
+  if (e == cudaSuccess) e = proj_configure();
+  if (e != cudaSuccess) return e;
+  ProjArgs a{};
+  a.M = static_cast<int>(M);
+  a.n = n;
+  a.d = d;
+  a.ksplit = 1;
+  a.pos = pos;
+  a.n_cap = n_cap;
+  a.codes = codes;
+  a.scales = scales;
+  a.dev_err = dev_err;
   const int64_t tiles = ((M + kCedM - 1) / kCedM) * (D / kCedN);
   const dim3 grid(static_cast<unsigned>(std::min<int64_t>(tiles, device_sm_count())));
-  e = launch_pdl(ced_quant_kernel, grid, dim3(kCedThreads), sizeof(CedSmem), s, map_h, map_w,
-                 static_cast<int>(M), n, d, pos, n_cap, codes, scales, dev_err);
+  profile_begin(CSA2_KERNEL_CED, s);
+  e = launch_pdl(ced_quant_kernel, grid, dim3(kCedThreads), sizeof(CedSmem), s, map_h, map_w, a);
+  profile_end(CSA2_KERNEL_CED, s);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+size_t swa_replay_workspace_bytes(int B, int Wr, int d) {
+  const int64_t M = static_cast<int64_t>(B) * Wr;
+  return static_cast<size_t>(replay_ksplit(M, d)) * static_cast<size_t>(M) * D * sizeof(float);
+}
+
+cudaError_t launch_swa_replay(const void* h, const void* w, int B, int Wr, int d, const int32_t* N,
+                              uint8_t* swa, float* swa_scale, int W, void* ws, int32_t* dev_err,
+                              cudaStream_t s) {
+  const int64_t M = static_cast<int64_t>(B) * Wr;
+  CUtensorMap map_h, map_w;
+  cudaError_t e = proj_tensor_maps(h, w, M, d, &map_h, &map_w);
+  if (e == cudaSuccess) e = proj_configure();
+  if (e != cudaSuccess) return e;
+  const int ksplit = replay_ksplit(M, d);
+  ProjArgs a{};
+  a.M = static_cast<int>(M);
+  a.n = Wr;
+  a.d = d;
+  a.ksplit = ksplit;
+  a.part = static_cast<float*>(ws);
+  a.dev_err = dev_err;
+  const int64_t tiles = ((M + kCedM - 1) / kCedM) * (D / kCedN) * ksplit;
+  const dim3 grid(static_cast<unsigned>(std::min<int64_t>(tiles, device_sm_count())));
+  profile_begin(CSA2_KERNEL_REPLAY, s);
+  e = launch_pdl(replay_proj_kernel, grid, dim3(kCedThreads), sizeof(CedSmem), s, map_h, map_w, a);
+  count_launches(1);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e == cudaSuccess) {
+    const dim3 grid2(static_cast<unsigned>((M + kReplayWarps - 1) / kReplayWarps));
+    e = launch_pdl(replay_swa_kernel, grid2, dim3(kReplayWarps * 32), 0, s,
+                   static_cast<const float*>(ws), ksplit, static_cast<int>(M), Wr, N, swa,
+                   swa_scale, W, dev_err);
+    count_launches(1);
+    if (e == cudaSuccess) e = cudaGetLastError();
+  }
+  profile_end(CSA2_KERNEL_REPLAY, s);
+  return e;
 }
 
 }  // namespace csa2

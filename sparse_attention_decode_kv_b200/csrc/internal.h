@@ -54,4 +54,11 @@ cudaError_t launch_ced_quant(const void* h, const void* w, int B, int n, int d, 
                              int n_cap, uint8_t* codes, uint8_t* scales, int32_t* dev_err,
                              cudaStream_t s);
 
+// SWA bounded replay: split-K tcgen05 projection of the window rows, then bf16 rounding and the
+// SWA codec into the ring.
+size_t swa_replay_workspace_bytes(int B, int Wr, int d);
+cudaError_t launch_swa_replay(const void* h, const void* w, int B, int Wr, int d, const int32_t* N,
+                              uint8_t* swa, float* swa_scale, int W, void* ws, int32_t* dev_err,
+                              cudaStream_t s);
+
 }  // namespace csa2

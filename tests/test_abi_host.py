@@ -43,7 +43,7 @@ def test_status_strings_and_version(L):
     assert csa2.status_string(0) == "CSA2_OK"
     for s in (-1, -2, -3, -4, -5, -6):
         assert csa2.status_string(s).startswith("CSA2_ERR")
-    assert L.csa2_abi_version() == 2
+    assert L.csa2_abi_version() == 3
     assert csa2.launch_count() >= 0
 
 
@@ -108,6 +108,67 @@ def test_ced_projection_rejects_bad_arguments(L):
     assert ced(L, d=65600) == UNSUPPORTED
     assert ced(L, B=4096, n=1 << 15) == UNSUPPORTED  # more than 2^26 tokens
     assert ced(L, n=0) == OK                         # nothing to do: no launch
+
+
+def replay(L, ws_bytes=1 << 30, **kw):
+    a = dict(h=FAKE, w=FAKE, B=2, Wr=128, d=256, N=FAKE, swa=FAKE, swa_scale=FAKE, W=128, ws=FAKE,
+             dev_err=None)
+    a.update(kw)
+    return L.csa2_swa_replay(P(a["h"]), P(a["w"]), a["B"], a["Wr"], a["d"], P(a["N"]), P(a["swa"]),
+                             P(a["swa_scale"]), a["W"], P(a["ws"]), ws_bytes, P(a["dev_err"]), None)
+
+
+def test_swa_replay_rejects_bad_arguments(L):
+    assert replay(L, B=0) == INVALID
+    assert replay(L, Wr=-1) == INVALID
+    assert replay(L, Wr=129) == INVALID              # more window rows than ring slots
+    assert replay(L, W=0) == INVALID
+    assert replay(L, d=96) == INVALID                # not a multiple of 64
+    assert replay(L, h=0) == INVALID
+    assert replay(L, w=MIS) == INVALID
+    assert replay(L, N=0) == INVALID
+    assert replay(L, swa_scale=0) == INVALID
+    assert replay(L, dev_err=FAKE + 2) == INVALID
+    assert replay(L, d=65600) == UNSUPPORTED
+    assert replay(L, W=8192, Wr=8) == UNSUPPORTED
+    assert replay(L, ws_bytes=16) == WORKSPACE
+    assert replay(L, ws=0) == WORKSPACE
+    assert replay(L, Wr=0) == OK                      # nothing to do: no launch
+
+
+def test_swa_replay_workspace_size(L):
+    # 2 x 128 rows = 2 token tiles x 2 channel halves = 4 tiles; the d-slices split 37 ways
+    # (148 / 4) but never more than d / 64
+    assert csa2.swa_replay_workspace_bytes(2, 128, 4096) == 37 * 256 * 512 * 4
+    assert csa2.swa_replay_workspace_bytes(2, 128, 256) == 4 * 256 * 512 * 4
+    assert csa2.swa_replay_workspace_bytes(8, 4096, 64) == 1 * 8 * 4096 * 512 * 4
+    assert csa2.swa_replay_workspace_bytes(0, 128, 256) == 0
+    assert csa2.swa_replay_workspace_bytes(2, 128, 100) == 0
+
+
+def cache_copy(L, fn, N=(5, 7), **kw):
+    a = dict(dc=FAKE, ds=FAKE, di=FAKE, B=2, n_cap=64, n_host=32, hc=FAKE, hs=FAKE, hi=FAKE)
+    a.update(kw)
+    n = (ctypes.c_int32 * len(N))(*N)
+    if fn == "restore":
+        return L.csa2_cache_restore(P(a["hc"]), P(a["hs"]), P(a["hi"]), a["B"], a["n_host"], n,
+                                    a["n_cap"], P(a["dc"]), P(a["ds"]), P(a["di"]), None)
+    return L.csa2_cache_persist(P(a["dc"]), P(a["ds"]), P(a["di"]), a["B"], a["n_cap"], n,
+                                a["n_host"], P(a["hc"]), P(a["hs"]), P(a["hi"]), None)
+
+
+@pytest.mark.parametrize("fn", ["restore", "persist"])
+def test_cache_copies_reject_bad_arguments(L, fn):
+    assert cache_copy(L, fn, B=0) == INVALID
+    assert cache_copy(L, fn, n_cap=60) == INVALID    # not a multiple of 8
+    assert cache_copy(L, fn, n_host=-1) == INVALID
+    assert cache_copy(L, fn, N=(5, 33)) == INVALID   # more rows than the host layout holds
+    assert cache_copy(L, fn, N=(5, 70), n_host=128) == INVALID  # more than the cache holds
+    assert cache_copy(L, fn, N=(-1, 3)) == INVALID
+    assert cache_copy(L, fn, dc=0) == INVALID
+    assert cache_copy(L, fn, hs=MIS) == INVALID
+    assert cache_copy(L, fn, hi=0) == INVALID        # keys on one side only
+    assert cache_copy(L, fn, di=0, hi=0, B=5000, N=(0,) * 5000) == UNSUPPORTED
 
 
 def index_full(L, ws_bytes=None, **kw):
