@@ -776,7 +776,7 @@ def replay_cpu_baseline(hc, hs, hi, hwin, w, N):
     hb = hwin[:1].contiguous().view(torch.int16).numpy().view(np.uint16)
     wb = w.contiguous().view(torch.int16).numpy().view(np.uint16)
     t0 = time.perf_counter()
-    for src in (hc, hs, hi):
+    for src in (hc, hs, hi.view(torch.int16)):
         np.copy(src.numpy())
     t_copy = time.perf_counter() - t0
     swa = np.zeros((1, W, 512), np.uint8)

@@ -353,6 +353,7 @@ __global__ void __launch_bounds__(kCedThreads, 1)
 
 // One warp per window row: sum of the partials (split 0 first), bf16 rounding, SWA codec.
 constexpr int kReplayWarps = 8;
+constexpr int kReplaySumBatch = 4;  // partial rows requested at once per lane
 __global__ void __launch_bounds__(kReplayWarps * 32)
     replay_swa_kernel(const float* __restrict__ part, int ksplit, int M, int Wr,
                       const int32_t* __restrict__ N, uint8_t* __restrict__ swa,
@@ -373,18 +374,35 @@ __global__ void __launch_bounds__(kReplayWarps * 32)
   float v[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) v[k] = 0.0f;
-  for (int ks = 0; ks < ksplit; ++ks) {
-    const float4* src =
-        reinterpret_cast<const float4*>(part + (static_cast<int64_t>(ks) * M + row) * D + 16 * lane);
+  const float* base = part + static_cast<int64_t>(row) * D + 16 * lane;
+  const int64_t split_stride = static_cast<int64_t>(M) * D;
+  int ks = 0;
+  for (; ks + kReplaySumBatch <= ksplit; ks += kReplaySumBatch) {  // loads of a batch in flight
+    float4 f[kReplaySumBatch][4];
+#pragma unroll
+    for (int u = 0; u < kReplaySumBatch; ++u)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        f[u][q] = __ldg(reinterpret_cast<const float4*>(base + (ks + u) * split_stride) + q);
+#pragma unroll
+    for (int u = 0; u < kReplaySumBatch; ++u)  // added in split order
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        v[4 * q] += f[u][q].x;
+        v[4 * q + 1] += f[u][q].y;
+        v[4 * q + 2] += f[u][q].z;
+        v[4 * q + 3] += f[u][q].w;
+      }
+  }
+  for (; ks < ksplit; ++ks)
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float4 f = __ldg(src + q);
+      const float4 f = __ldg(reinterpret_cast<const float4*>(base + ks * split_stride) + q);
       v[4 * q] += f.x;
       v[4 * q + 1] += f.y;
       v[4 * q + 2] += f.z;
       v[4 * q + 3] += f.w;
     }
-  }
 #pragma unroll
   for (int k = 0; k < 16; ++k) v[k] = __bfloat162float(__float2bfloat16_rn(v[k]));
   uint32_t e[4];
