@@ -10,10 +10,15 @@ algorithmic bytes (indexer keys read + gathered MXFP4 codes and scales + FP8 SWA
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
   python bench.py --ced [--steps K] [--warmup W]
+  python bench.py --replay [--replay-n N] [--steps K] [--warmup W]
 
 --ced measures the CED KV projection with the MXFP4 epilogue instead (8 x 4,096 new tokens,
 hidden size 4,096: a tensor-core-bound GEMM), reported in TFLOP/s against the measured bf16
 tensor peak.
+--replay measures the SWA bounded replay restore of 8 persisted sequences of N tokens (default
+1,048,576): the host-to-device reload of their MXFP4 KV and indexer keys from pinned memory
+(reported against a plain pinned copy of the same bytes) and the replay of their FP8 SWA rings
+from the last 128 tokens' hidden states (d = 4,096; tcgen05 projection, TFLOP/s).
 
 With --gpus N > 1 run under torchrun: every rank decodes its own batch (data parallel, no
 collective on the data path); the step time is the max over ranks.
@@ -60,6 +65,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--replay", action="store_true",
                     help="measure the SWA bounded replay restore (host reload + ring replay)")
+    ap.add_argument("--replay-n", type=int, default=1 << 20,
+                    help="tokens per restored sequence for --replay (default 1,048,576)")
     ap.add_argument("--ced", action="store_true",
                     help="measure the CED KV projection with the MXFP4 epilogue instead")
     ap.add_argument("--breakdown", action="store_true",
@@ -760,7 +767,7 @@ def run_ced(args, world, rank, local):
     if rank == 0:
         print(json.dumps(line), flush=True)
 
-REPLAY_METRIC = ("SWA bounded replay: sequence restores/s (1M-token prefix: host->HBM reload of the "
+REPLAY_METRIC = ("SWA bounded replay: sequence-batch restores/s (8 prefixes: host->HBM reload of the "
                  "MXFP4 KV + indexer keys, FP8 SWA ring replayed from the last 128 tokens), 1 B200")
 REPLAY_SHAPE = dict(B=8, N=1 << 20, W=128, d=4096)
 
@@ -800,6 +807,9 @@ def run_replay(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     B, N, W, d = (REPLAY_SHAPE[k] for k in ("B", "N", "W", "d"))
+    N = int(args.replay_n)
+    if N < W or N % 8:
+        raise SystemExit("--replay-n must be a multiple of 8 and at least the window (128)")
     g = torch.Generator(device=dev).manual_seed(2000 + rank)
     stream = torch.cuda.current_stream(dev)
     # the persisted state: written once from device buffers through csa2_cache_persist
@@ -906,7 +916,7 @@ def run_replay(args, world, rank, local):
         "dtype": "u8 copies + bf16-in fp32-acc (fp8 out)", "data": "synthetic",
         "config": {"workload": f"swa-replay-restore-B{B}-N{N}-W{W}-d{d}", "sequences": B,
                    "tokens_per_sequence": N, "window": W, "d": d,
-                   "l2": "inputs larger than L2 (3.5 GB reloaded per step)",
+                   "l2": "inputs larger than L2 (%.2f GB reloaded per step)" % (reload_bytes / 1e9),
                    "parallelism": f"dp{world} (independent sequences)"},
         "reload": {"achieved_gbs": round(reload_bytes / (c_ms / 1e3) / 1e9, 1),
                    "peak_gbs": round(link_gbs, 1),
