@@ -11,10 +11,14 @@ algorithmic bytes (indexer keys read + gathered MXFP4 codes and scales + FP8 SWA
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
   python bench.py --ced [--steps K] [--warmup W]
   python bench.py --replay [--replay-n N] [--steps K] [--warmup W]
+  python bench.py --queries [--steps K] [--warmup W]
 
 --ced measures the CED KV projection with the MXFP4 epilogue instead (8 x 4,096 new tokens,
 hidden size 4,096: a tensor-core-bound GEMM), reported in TFLOP/s against the measured bf16
 tensor peak.
+--queries measures csa2_attend_queries on a prefill chunk: 8 sequences of 131,072 cached entries,
+512 query tokens each (4,096 queries), every query with its own 512 selected entries and its own
+causal window of 128 FP8 SWA rows; reported in queries/s and GB/s of gathered bytes.
 --replay measures the SWA bounded replay restore of 8 persisted sequences of N tokens (default
 1,048,576): the host-to-device reload of their MXFP4 KV and indexer keys from pinned memory
 (reported against a plain pinned copy of the same bytes) and the replay of their FP8 SWA rings
@@ -65,6 +69,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--replay", action="store_true",
                     help="measure the SWA bounded replay restore (host reload + ring replay)")
+    ap.add_argument("--queries", action="store_true",
+                    help="measure multi-query sparse attention (prefill / verification queries)")
     ap.add_argument("--replay-n", type=int, default=1 << 20,
                     help="tokens per restored sequence for --replay (default 1,048,576)")
     ap.add_argument("--ced", action="store_true",
@@ -767,6 +773,156 @@ def run_ced(args, world, rank, local):
     if rank == 0:
         print(json.dumps(line), flush=True)
 
+QUERIES_METRIC = ("multi-query sparse attention (prefill / verification): queries/s and achieved GB/s "
+                  "of gathered MXFP4 + FP8 SWA bytes, 1 B200")
+QUERIES_SHAPE = dict(B=8, N=131072, T=512, K=512, W=128)
+
+
+def queries_cpu_baseline(q, codes, scales, idx, swa, swsc, qseq, lo, ln, n_sample=320):
+    """The oracle's attention of a sample of the queries, scaled to queries/s."""
+    import numpy as np
+    import oracle
+    from oracle import build as oracle_build
+    oracle_build.build()
+    Q = q.shape[0]
+    pick = np.linspace(0, Q - 1, n_sample).astype(np.int64)
+    qb = q[pick].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    t0 = time.perf_counter()
+    for j, i in enumerate(pick):
+        b, a, n = int(qseq[i]), int(lo[i]), int(ln[i])
+        oracle.attend_seq(qb[j], 1.0, codes[b], scales[b], idx[i].astype(np.int64),
+                          swa[b, a:a + n], swsc[b, a:a + n], n)
+    sec = time.perf_counter() - t0
+    return {"value": round(n_sample / sec, 3), "unit": "queries/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n_sample} of {Q} queries, evenly spaced ({sec:.2f} s)",
+            "seconds": round(sec, 2)}
+
+
+def run_queries(args, world, rank, local):
+    import numpy as np
+    import sparse_attention_decode_kv_b200 as csa2
+    from sparse_attention_decode_kv_b200 import build as csa2_build
+    if rank == 0:
+        csa2_build.build()
+    barrier(world)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    B, N, T, K, W = (QUERIES_SHAPE[k] for k in ("B", "N", "T", "K", "W"))
+    Q = B * T
+    g = torch.Generator(device=dev).manual_seed(3000 + rank)
+    stream = torch.cuda.current_stream(dev)
+    # the prefix: N cached entries per sequence, appended in chunks through the library
+    cache = csa2.Cache(B, N, 0, device=dev)
+    chunk = 16384
+    for c0 in range(0, N, chunk):
+        x = torch.randn(B, chunk, 512, device=dev, generator=g).to(torch.bfloat16)
+        csa2.append_quant(x, None, torch.full((B,), c0, dtype=torch.int32, device=dev),
+                          cache.codes, cache.scales, None)
+    # FP8 SWA rows of every position (E4M3 magnitudes below 448: bytes 0x00..0x7E per sign)
+    mag = torch.randint(0, 0x7F, (B, N, 512), dtype=torch.uint8, device=dev, generator=g)
+    sgn = torch.randint(0, 2, (B, N, 512), dtype=torch.uint8, device=dev, generator=g) << 7
+    swa = mag | sgn
+    del mag, sgn
+    swsc = torch.rand(B, N, device=dev, generator=g) * 0.01 + 1e-4
+    # query t of sequence b is the prompt token at position p = N - T + t: its selection is K
+    # positions below p (sorted), its window the rows max(0, p - W + 1) .. p
+    qseq = torch.arange(B, device=dev, dtype=torch.int32).repeat_interleave(T)
+    pos = (N - T + torch.arange(T, device=dev)).repeat(B)
+    idx = (torch.rand(Q, K, device=dev, generator=g) * pos[:, None]).to(torch.int32).sort(1).values
+    lo = (pos - W + 1).clamp(min=0).to(torch.int32)
+    ln = (pos - lo + 1).to(torch.int32)
+    q = (torch.randn(Q, 16, 512, device=dev, generator=g) / 512 ** 0.5).to(torch.bfloat16)
+    out = torch.empty(Q, 16, 512, device=dev)
+    lse = torch.empty(Q, 16, device=dev)
+    ws = csa2.workspace(csa2.attend_workspace_bytes(Q, K, W), dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    Nt = torch.full((B,), N, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+
+    def step():
+        csa2.attend_queries(q, 1.0, cache.codes, cache.scales, Nt, qseq, idx, swa, swsc, lo, ln, W,
+                            out, lse, ws, err)
+
+    Ks, Wu = args.steps, args.warmup
+    launches0 = csa2.launch_count()
+    step()
+    torch.cuda.synchronize()
+    per_step_launches = csa2.launch_count() - launches0
+    for _ in range(Wu):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(Ks):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = max_over_ranks(world, t0.elapsed_time(t1), dev) / Ks
+    if int(err.item()):
+        raise RuntimeError(f"device error flags {int(err.item()):#x} during the benchmark")
+    per_query = K * 288 + W * 516
+    byts = Q * per_query
+    gbs = byts / (ms / 1e3) / 1e9
+    peak, peak_kind = measured_peak()
+    e2e = None
+    if not args.no_e2e:
+        q_h = q.cpu().pin_memory()
+        idx_h = idx.cpu().pin_memory()
+        out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        ke = max(1, min(Ks, 20))
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(ke):
+            q.copy_(q_h, non_blocking=True)
+            idx.copy_(idx_h, non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / ke
+        e2e = {"value": round(world * Q / (e_ms / 1e3), 1), "unit": "queries/s",
+               "h2d_bytes_per_step": q.numel() * 2 + idx.numel() * 4,
+               "d2h_bytes_per_step": out.numel() * 4}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = queries_cpu_baseline(q.cpu(), cache.codes.cpu().numpy(), cache.scales.cpu().numpy(),
+                                   idx.cpu().numpy(), swa.cpu().numpy(), swsc.cpu().numpy(),
+                                   qseq.cpu().numpy(), lo.cpu().numpy(), ln.cpu().numpy())
+    line = {
+        "metric": QUERIES_METRIC, "value": round(world * Q / (ms / 1e3), 1), "unit": "queries/s",
+        "n_gpus": world, "steps": Ks, "warmup": Wu, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp16-in fp32-acc (mxfp4 + fp8 cache)", "data": "synthetic",
+        "config": {"workload": f"prefill-queries-B{B}-N{N}-T{T}-K{K}-W{W}", "queries": Q,
+                   "sequences": B, "cached_entries": N, "K": K, "W": W,
+                   "l2": "inputs larger than L2 (%.0f MB of MXFP4 cache, %.0f MB of SWA rows)"
+                         % (cache.codes.numel() * 1.125 / 1e6, swa.numel() * 1.0078 / 1e6),
+                   "parallelism": f"dp{world} (independent sequences)"},
+        "achieved_gbs": round(gbs, 1),
+        "roofline": {"kernel": "attend_kernel (multi-query)", "bound": "hbm",
+                     "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4), "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": byts,
+                     "algorithmic_bytes_per_query": per_query,
+                     "launch_ms": round(ms, 4), "traffic": None,
+                     "note": "algorithmic bytes count every query's gathered rows; neighbouring "
+                             "queries share window rows, which L2 serves"},
+        "gpu_launches": per_step_launches * Ks,
+        "clocks": clocks.summary(),
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 REPLAY_METRIC = ("SWA bounded replay: sequence-batch restores/s (8 prefixes: host->HBM reload of the "
                  "MXFP4 KV + indexer keys, FP8 SWA ring replayed from the last 128 tokens), 1 B200")
 REPLAY_SHAPE = dict(B=8, N=1 << 20, W=128, d=4096)
@@ -949,6 +1105,8 @@ def main():
             run_ced(args, world, rank, local)
         elif args.replay and args.impl == "ours":
             run_replay(args, world, rank, local)
+        elif args.queries and args.impl == "ours":
+            run_queries(args, world, rank, local)
         elif args.impl == "reference":
             run_reference(args, world, rank, local)
         else:

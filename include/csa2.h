@@ -38,6 +38,12 @@
  *   - Workspaces: query the byte count with the matching *_workspace_bytes function; pass a device
  *     buffer of at least that many bytes. Contents need no initialisation.
  *   - Calls that share a workspace must not overlap on the GPU.
+ *   - Kernels after the first of a call are launched with programmatic dependent launch: each may
+ *     start while the kernel before it on the stream finishes, and waits for it before reading
+ *     anything a kernel can have produced. Kernels outside this library never trigger that early
+ *     start, so their results are complete before a call begins. The attention kernels read q
+ *     before the wait, since no kernel of this library writes q: q must not alias memory that the
+ *     preceding calls of this library on the stream write.
  */
 #ifndef CSA2_H
 #define CSA2_H

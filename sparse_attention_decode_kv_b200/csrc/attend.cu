@@ -101,6 +101,47 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, c = lane & 3;
   const int b = blockIdx.x, split = blockIdx.y, nsplit = gridDim.y;  // b on x: up to 2^31 - 1
+  // ---- q -> fp16 with a per-head power-of-two scale (16 threads per head, 32 dims each). No
+  // kernel of this library writes q, so this runs before the wait on the preceding kernel and
+  // overlaps its tail.
+  {
+    const int h = tid >> 4, r = tid & 15;
+    const uint4* src = reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * HQ + h) * D) +
+                       4 * r;
+    uint4 u[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u[k] = __ldg(src + k);
+    float amax = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t w4[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w4[e])), fabsf(bf16hi(w4[e]))));
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+    const int eh = amax > 0.0f ? ilog2f(amax) : 0;
+    const float up = pow2f(14 - eh);
+    if (r == 0) {
+      sm.q_unscale[h] = pow2f(eh - 14) * softmax_scale;
+      sm.m_run[h] = -INFINITY;
+      sm.l_run[h] = 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t w4[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+      uint32_t h2[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        __half2 hv = __floats2half2_rn(bf16lo(w4[e]) * up, bf16hi(w4[e]) * up);
+        h2[e] = *reinterpret_cast<uint32_t*>(&hv);
+      }
+      *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(sm.q) + swz1024(h, 4 * r + k)) =
+          make_uint4(h2[0], h2[1], h2[2], h2[3]);
+    }
+  }
+
   pdl_wait();
   pdl_launch_dependents();
 
@@ -140,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
 
-  // the first tile's indices load before the query prologue so the two latencies overlap
+  // the first tile's indices (possibly written by the preceding kernel)
   int pos_first[4] = {-1, -1, -1, -1};
   if (t_begin < t_end && t_begin < tiles_idx) {
 #pragma unroll
@@ -148,45 +189,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int item = pass * 16 + (tid >> 4);
       if (item < min(kTile, K - t_begin * kTile))
         pos_first[pass] = __ldg(idx + static_cast<int64_t>(b) * K + t_begin * kTile + item);
-    }
-  }
-
-  // ---- q -> fp16 with a per-head power-of-two scale (16 threads per head, 32 dims each)
-  {
-    const int h = tid >> 4, r = tid & 15;
-    const uint4* src = reinterpret_cast<const uint4*>(q + (static_cast<int64_t>(b) * HQ + h) * D) +
-                       4 * r;
-    uint4 u[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) u[k] = __ldg(src + k);
-    float amax = 0.0f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint32_t w4[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w4[e])), fabsf(bf16hi(w4[e]))));
-    }
-#pragma unroll
-    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-    const int eh = amax > 0.0f ? ilog2f(amax) : 0;
-    const float up = pow2f(14 - eh);
-    if (r == 0) {
-      sm.q_unscale[h] = pow2f(eh - 14) * softmax_scale;
-      sm.m_run[h] = -INFINITY;
-      sm.l_run[h] = 0.0f;
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint32_t w4[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
-      uint32_t h2[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        __half2 hv = __floats2half2_rn(bf16lo(w4[e]) * up, bf16hi(w4[e]) * up);
-        h2[e] = *reinterpret_cast<uint32_t*>(&hv);
-      }
-      *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(sm.q) + swz1024(h, 4 * r + k)) =
-          make_uint4(h2[0], h2[1], h2[2], h2[3]);
     }
   }
 
