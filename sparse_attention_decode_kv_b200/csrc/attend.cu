@@ -68,6 +68,24 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // Row of 64 16-byte chunks. The low three chunk bits are XORed with the row's low bits (the 8 rows
 // of an ldmatrix read at one chunk fall in 8 distinct bank groups) and with the chunk's own bits
 // 3..5 (the chunks 4r + k, r = 0..7, that 8 threads store at once also fall in 8 distinct groups).
+// Four bytes of E2M1 pairs -> four half2 (byte j -> o[j], low nibble in .x). The byte unpack
+// leaves the choice of byte operands to the compiler instead of a shift and mask per byte.
+__device__ __forceinline__ void e2m1x8_to_h2x4(uint32_t w, uint32_t (&o)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+      : "r"(w));
+}
+
+// Four E4M3 bytes -> two half2 (bytes 0, 1 -> o[0]; bytes 2, 3 -> o[1]). Exact.
+__device__ __forceinline__ void e4m3x4_to_h2x2(uint32_t w, uint32_t (&o)[2]) {
+  asm("{\n\t.reg .b16 h0, h1;\n\tmov.b32 {h0, h1}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, h0;\n\tcvt.rn.f16x2.e4m3x2 %1, h1;\n\t}"
+      : "=r"(o[0]), "=r"(o[1])
+      : "r"(w));
+}
+
 __device__ __forceinline__ uint32_t swz1024(int row, int chunk) {
   return static_cast<uint32_t>(row * 1024 + ((chunk ^ (row & 7) ^ ((chunk >> 3) & 7)) << 4));
 }
@@ -223,8 +241,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     // All index loads, then all row loads, then the conversions: two memory round trips.
     {
       const int r = tid & 15;
+      // item = 16 pass + tid / 16 has the row bits of tid / 16, so each pass's store address is
+      // the pass's 16 KiB row block plus one of four per-thread offsets
       unsigned char* vrow = reinterpret_cast<unsigned char*>(sm.v);
       if (!is_swa) {
+        uint32_t off[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) off[k] = swz1024(tid >> 4, 4 * r + k);
         int pos[4];
 #pragma unroll
         for (int pass = 0; pass < 4; ++pass) {
@@ -257,22 +280,24 @@ __global__ void __launch_bounds__(kThreads, 2)
           const uint32_t s01 = e4m3x2_to_h2(sw[pass]);  // .x: channels 32r..+15, .y: the next 16
           const uint32_t slo = __byte_perm(s01, 0, 0x1010), shi = __byte_perm(s01, 0, 0x3232);
           const uint32_t cws[4] = {cw[pass].x, cw[pass].y, cw[pass].z, cw[pass].w};
-          uint32_t hv[16];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const uint32_t byte = (cws[k >> 2] >> (8 * (k & 3))) & 0xFFu;
-            hv[k] = h2_mul(e2m1x2_to_h2(byte), k < 8 ? slo : shi);
+          for (int k = 0; k < 4; ++k) {  // word k: channels 32r + 8k .. + 7
+            uint32_t hv[4];
+            e2m1x8_to_h2x4(cws[k], hv);
+            const uint32_t sk = k < 2 ? slo : shi;
+            *reinterpret_cast<uint4*>(vrow + pass * (16 * 1024) + off[k]) =
+                make_uint4(h2_mul(hv[0], sk), h2_mul(hv[1], sk), h2_mul(hv[2], sk), h2_mul(hv[3], sk));
           }
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<uint4*>(vrow + swz1024(item, 4 * r + k)) =
-                make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
           if (r == 0) {
             sm.item_valid[item] = valid;
             sm.item_scale[item] = 1.0f;
           }
         }
       } else {
+        uint32_t off[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)  // chunks 2r, 2r + 1, 32 + 2r, 33 + 2r
+          off[k] = swz1024(tid >> 4, 2 * r + (k & 1) + 32 * (k >> 1));
         uint4 e[4][2];
         float iscale[4];
 #pragma unroll
@@ -294,16 +319,14 @@ __global__ void __launch_bounds__(kThreads, 2)
           const bool valid = item < count && base + item < sl;
           const uint32_t ew[8] = {e[pass][0].x, e[pass][0].y, e[pass][0].z, e[pass][0].w,
                                   e[pass][1].x, e[pass][1].y, e[pass][1].z, e[pass][1].w};
-          uint32_t hv[16];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            hv[2 * k] = e4m3x2_to_h2(ew[k] & 0xFFFFu);
-            hv[2 * k + 1] = e4m3x2_to_h2(ew[k] >> 16);
+          for (int k = 0; k < 4; ++k) {
+            uint32_t h0[2], h1[2];
+            e4m3x4_to_h2x2(ew[2 * k], h0);
+            e4m3x4_to_h2x2(ew[2 * k + 1], h1);
+            *reinterpret_cast<uint4*>(vrow + pass * (16 * 1024) + off[k]) =
+                make_uint4(h0[0], h0[1], h1[0], h1[1]);
           }
-#pragma unroll
-          for (int k = 0; k < 4; ++k)  // chunks 2r, 2r + 1, 32 + 2r, 33 + 2r
-            *reinterpret_cast<uint4*>(vrow + swz1024(item, 2 * r + (k & 1) + 32 * (k >> 1))) =
-                make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
           if (r == 0) {
             sm.item_valid[item] = valid;
             sm.item_scale[item] = iscale[pass];
