@@ -234,6 +234,23 @@ class ReuseAttendWorkload:
     seed: int = 4
 
 
+# The throughput sweep's Reuse-mode attention: batch 1, 8, 64 and 256 over N = 131,072.
+REUSE_SWEEP = tuple(ReuseAttendWorkload(f"reuse-attend-B{B}-N131072", B=B) for B in (1, 8, 64, 256))
+
+
+def reuse_kv_chunk(wl: ReuseAttendWorkload, b: int, c: int, device="cpu") -> torch.Tensor:
+    """Main-KV rows [c*CHUNK, min((c+1)*CHUNK, N)) of sequence b, N(0,1) bf16 [rows, 512]."""
+    rows = min(CHUNK, wl.N - c * CHUNK)
+    g = gen(device, wl.seed, "kv", b, c)
+    return torch.randn(rows, D, generator=g, device=device).to(torch.bfloat16)
+
+
+def reuse_queries(wl: ReuseAttendWorkload, device="cpu") -> torch.Tensor:
+    """q [B, 16, 512] bf16, N(0,1)/sqrt(512)."""
+    g = gen(device, wl.seed, "q", 0)
+    return (torch.randn(wl.B, HQ, D, generator=g, device=device) / math.sqrt(D)).to(torch.bfloat16)
+
+
 def reuse_indices(wl: ReuseAttendWorkload, device="cpu") -> torch.Tensor:
     out = torch.empty(wl.B, wl.K, dtype=torch.int32)
     for b in range(wl.B):
