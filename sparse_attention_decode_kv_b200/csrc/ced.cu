@@ -376,6 +376,225 @@ __global__ void __launch_bounds__(kCedThreads, 1)
   proj_body<kEpiF32Partial>(&tm_h, &tm_w, &tm_w, a);  // no half-width tiles
 }
 
+// ---------------------------------------------------------------------------- CTA-pair kernel
+//
+// ced_pair_kernel: the same projection and MXFP4 epilogue with the MMA shared by the two CTAs of a
+// cluster (tcgen05 cta_group::2). A pair tile is 256 tokens x 256 channels: CTA r of the pair
+// loads its 128 token rows of h and channels 128 r .. 128 r + 127 of the tile's w rows (16 KiB
+// each per 64-wide d-slice), the leader issues M 256 x N 256 x K 16 MMAs that read both CTAs'
+// stages, and each CTA's tensor memory receives its own 128 rows x 256 channels. Per unit of MMA
+// work each CTA streams a third less than a CTA of ced_quant_kernel (32 instead of 48 KiB per
+// d-slice), and the freed shared memory holds six stages instead of four.
+//   warp 0, one thread  TMA producer (both CTAs): loads this CTA's halves; the copies of both
+//                       CTAs complete on the leader's stage barrier, whose producer alone posts the
+//                       pair's byte count.
+//   warp 1, one thread  MMA issuer (leader only): waits for a stage, issues four pair MMAs,
+//                       commits to the stage's empty barrier in both CTAs; after a tile, commits
+//                       to the accumulator-full barrier in both CTAs. Warp 1 of both CTAs
+//                       allocates and frees the pair's tensor memory.
+//   warps 2..5          epilogue (both CTAs): as in ced_quant_kernel on this CTA's rows, then one
+//                       arrival per warp on the leader's accumulator-empty barrier (8 per tile).
+constexpr int kPairStages = 6;
+constexpr int kPairTile = 128 * kCedK * 2;  // 16 KiB: 128 rows of a 64-wide bf16 d-slice
+constexpr uint32_t kPairIdesc = umma_idesc_bf16_f32(2 * kCedM, kCedN);
+
+struct __align__(1024) CedPairSmem {
+  uint8_t a[kPairStages][kPairTile];
+  uint8_t b[kPairStages][kPairTile];
+  uint64_t full[kPairStages];   // leader: both CTAs' copies of the stage have landed
+  uint64_t empty[kPairStages];  // each CTA: the pair MMAs have read the stage
+  uint64_t acc_full[2];         // each CTA: the accumulator is complete
+  uint64_t acc_empty[2];        // leader: the 8 epilogue warps of the pair have read it out
+  uint64_t drain;               // each CTA: every pair MMA has completed
+  uint32_t tmem_base;
+  int abort;
+};
+
+static_assert(sizeof(CedPairSmem) <= 227 * 1024, "ced_pair_kernel shared memory");
+
+__global__ void __launch_bounds__(kCedThreads, 1)
+    ced_pair_kernel(const __grid_constant__ CUtensorMap tm_h,
+                    const __grid_constant__ CUtensorMap tm_w_half, const ProjArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  CedPairSmem& sm = *reinterpret_cast<CedPairSmem*>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
+  const int M = a.M, n = a.n;
+  const int nk = a.d / kCedK;
+  int32_t* dev_err = a.dev_err;
+  const int tiles = ((M + 2 * kCedM - 1) / (2 * kCedM)) * (D / kCedN);
+  const int my_tiles = tiles > pair ? (tiles - 1 - pair) / npairs + 1 : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int c = 0; c < 2; ++c) {
+      mbar_init(&sm.acc_full[c], 1);
+      mbar_init(&sm.acc_empty[c], 2 * kCedEpiWarps);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&sm.tmem_base, kCedTmemCols);
+    tmem_relinquish_pair();
+  }
+  tcgen05_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before either signals the other's
+  tcgen05_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+  pdl_wait();  // h, w and pos may be written by the preceding kernel
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int it = 0;
+      for (int j = 0; j < my_tiles && !*abort; ++j) {
+        const int t = pair + j * npairs;
+        const int m0 = (t >> 1) * (2 * kCedM) + static_cast<int>(rank) * kCedM;
+        const int n0 = (t & 1) * kCedN + static_cast<int>(rank) * kCedNHalf;
+        for (int kc = 0; kc < nk; ++kc, ++it) {
+          const int s = it % kPairStages;
+          if (it >= kPairStages &&
+              !bounded_wait(&sm.empty[s], static_cast<uint32_t>(((it / kPairStages) & 1) ^ 1), abort)) {
+            if (!*abort) flag_error(dev_err, CSA2_DEVERR_TIMEOUT);
+            *abort = 1;
+            break;
+          }
+          const uint32_t full_leader = mapa_shared(smem_u32(&sm.full[s]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], 2 * 2 * kPairTile);
+          tma_load_2d_pair(sm.a[s], &tm_h, full_leader, kc * kCedK, m0);
+          tma_load_2d_pair(sm.b[s], &tm_w_half, full_leader, kc * kCedK, n0);
+        }
+      }
+      // the leader's stage barriers count both CTAs' copies: its drain covers the pair's
+      if (rank == 0)
+        for (int q = max(0, it - kPairStages); q < it; ++q)
+          if (!mbar_wait(&sm.full[q % kPairStages], static_cast<uint32_t>((q / kPairStages) & 1)))
+            flag_error(dev_err, CSA2_DEVERR_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------------------- MMA issuer
+    if (lane == 0 && rank == 0) {
+      int it = 0;
+      for (int j = 0; j < my_tiles && !*abort; ++j) {
+        const int acc = j & 1;
+        if (j >= 2 &&
+            !bounded_wait(&sm.acc_empty[acc], static_cast<uint32_t>(((j >> 1) & 1) ^ 1), abort)) {
+          if (!*abort) flag_error(dev_err, CSA2_DEVERR_TIMEOUT);
+          *abort = 1;
+          break;
+        }
+        tcgen05_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kCedN);
+        bool ok = true;
+        for (int kc = 0; kc < nk; ++kc, ++it) {
+          const int s = it % kPairStages;
+          if (!bounded_wait(&sm.full[s], static_cast<uint32_t>((it / kPairStages) & 1), abort)) {
+            if (!*abort) flag_error(dev_err, CSA2_DEVERR_TIMEOUT);
+            *abort = 1;
+            ok = false;
+            break;
+          }
+          tcgen05_fence_after();
+          const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
+#pragma unroll
+          for (int k4 = 0; k4 < kCedK / 16; ++k4)
+            umma_bf16_pair(d_tmem, umma_desc_k128(a0 + 32 * k4), umma_desc_k128(b0 + 32 * k4),
+                           kPairIdesc, (kc | k4) != 0 ? 1u : 0u);
+          const uint32_t e = smem_u32(&sm.empty[s]);
+          umma_commit_pair(mapa_shared(e, 0));  // both CTAs may refill the stage
+          umma_commit_pair(mapa_shared(e, 1));
+        }
+        const uint32_t f = smem_u32(&sm.acc_full[acc]);
+        umma_commit_pair(mapa_shared(f, 0));
+        umma_commit_pair(mapa_shared(f, 1));
+        if (!ok) break;
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;
+    const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&sm.acc_empty[0]), 0);
+    const uint32_t acc_empty_leader1 = mapa_shared(smem_u32(&sm.acc_empty[1]), 0);
+    for (int j = 0; j < my_tiles; ++j) {
+      const int acc = j & 1;
+      const int t = pair + j * npairs;
+      const int m0 = (t >> 1) * (2 * kCedM) + static_cast<int>(rank) * kCedM;
+      const int n0 = (t & 1) * kCedN;
+      const bool ok = __all_sync(0xFFFFFFFFu,
+                                 bounded_wait(&sm.acc_full[acc], static_cast<uint32_t>((j >> 1) & 1), abort));
+      if (!ok) {
+        if (lane == 0 && !*abort) flag_error(dev_err, CSA2_DEVERR_TIMEOUT);
+        break;
+      }
+      tcgen05_fence_after();
+      const int row = m0 + 32 * quarter + lane;
+      const uint32_t tbase =
+          tmem + static_cast<uint32_t>(acc * kCedN) + (static_cast<uint32_t>(32 * quarter) << 16);
+      int64_t dst = -1;
+      if (row < M) {
+        const int b = row / n, i = row - (row / n) * n;
+        const int64_t p = static_cast<int64_t>(__ldg(a.pos + b)) + i;
+        if (p >= 0 && p < a.n_cap) dst = static_cast<int64_t>(b) * a.n_cap + p;
+        else if (n0 == 0) flag_error(dev_err, CSA2_DEVERR_POS_RANGE);
+      }
+      uint32_t sc[16];
+#pragma unroll 1
+      for (int g = 0; g < kCedN / 16; ++g) {
+        uint32_t r[16];
+        tmem_ld16(tbase + static_cast<uint32_t>(16 * g), r);
+        tmem_wait_ld();
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+        uint32_t sb;
+        const uint2 cw = quantize_group_f32(v, sb);
+        sc[g] = sb;
+        if (dst >= 0) *reinterpret_cast<uint2*>(a.codes + dst * (D / 2) + n0 / 2 + 8 * g) = cw;
+      }
+      tcgen05_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
+      if (dst >= 0) {
+        uint4 packed;
+        packed.x = sc[0] | (sc[1] << 8) | (sc[2] << 16) | (sc[3] << 24);
+        packed.y = sc[4] | (sc[5] << 8) | (sc[6] << 16) | (sc[7] << 24);
+        packed.z = sc[8] | (sc[9] << 8) | (sc[10] << 16) | (sc[11] << 24);
+        packed.w = sc[12] | (sc[13] << 8) | (sc[14] << 16) | (sc[15] << 24);
+        *reinterpret_cast<uint4*>(a.scales + dst * (D / 16) + n0 / 16) = packed;
+      }
+    }
+  }
+  pdl_launch_dependents();
+  __syncthreads();
+  if (warp == 1) {
+    // every pair MMA must have completed before either CTA frees its tensor memory: the leader
+    // commits once more to a barrier used only here, in both CTAs
+    if (lane == 0) {
+      if (rank == 0) {
+        const uint32_t d = smem_u32(&sm.drain);
+        umma_commit_pair(mapa_shared(d, 0));
+        umma_commit_pair(mapa_shared(d, 1));
+      }
+      if (!bounded_wait(&sm.drain, 0u, nullptr)) flag_error(dev_err, CSA2_DEVERR_TIMEOUT);
+    }
+    __syncwarp();
+  }
+  tcgen05_fence_before();
+  cluster_sync();  // neither CTA leaves while the pair's MMAs or copies may use its memory
+  if (warp == 1) {
+    tcgen05_fence_after();
+    tmem_dealloc_pair(tmem, kCedTmemCols);
+  }
+}
+
 // One warp per window row: sum of the partials (split 0 first), bf16 rounding, SWA codec.
 constexpr int kReplayWarps = 8;
 constexpr int kReplaySumBatch = 4;  // partial rows requested at once per lane
@@ -481,6 +700,9 @@ cudaError_t proj_configure() {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(replay_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(sizeof(CedSmem)));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(ced_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(sizeof(CedPairSmem)));
     if (e != cudaSuccess) return e;
     g_ced_ready[dev] = 1;
   }
@@ -506,6 +728,26 @@ cudaError_t launch_ced_quant(const void* h, const void* w, int B, int n, int d, 
   cudaError_t e = proj_tensor_maps(h, w, M, d, &map_h, &map_w, &map_w_half);
   if (e == cudaSuccess) e = proj_configure();
   if (e != cudaSuccess) return e;
+  if (M >= 2 * kCedM) {  // CTA pairs: 256-token tiles, one cluster of 2 per tile slot
+    ProjArgs a{};
+    a.M = static_cast<int>(M);
+    a.n = n;
+    a.d = d;
+    a.ksplit = 1;
+    a.pos = pos;
+    a.n_cap = n_cap;
+    a.codes = codes;
+    a.scales = scales;
+    a.dev_err = dev_err;
+    const int64_t pair_tiles = ((M + 2 * kCedM - 1) / (2 * kCedM)) * (D / kCedN);
+    const int64_t pairs = std::min<int64_t>(pair_tiles, device_sm_count() / 2);
+    profile_begin(CSA2_KERNEL_CED, s);
+    e = launch_pdl_cluster(ced_pair_kernel, dim3(static_cast<unsigned>(2 * pairs)),
+                           dim3(kCedThreads), sizeof(CedPairSmem), s, 2, map_h, map_w_half, a);
+    profile_end(CSA2_KERNEL_CED, s);
+    count_launches(1);
+    return e != cudaSuccess ? e : cudaGetLastError();
+  }
   // A last wave that would fill at most half of the CTAs is cut into half-width tiles, which
   // then fill at most all of them and finish in about half the time.
   const int64_t tiles = ((M + kCedM - 1) / kCedM) * (D / kCedN);
