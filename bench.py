@@ -116,11 +116,11 @@ def scan_traffic_per_launch(wl):
 
 
 def ced_traffic_per_launch(tokens):
-    """DRAM bytes per CED launch from the committed ncu capture (profiles/ced_quant_traffic.json),
+    """DRAM bytes per CED launch from the committed ncu capture (profiles/ced_projection_traffic.json),
     scaled by token rows; None once the kernel's sources differ from the captured ones."""
     import hashlib
     try:
-        with open(os.path.join(ROOT, "profiles", "ced_quant_traffic.json")) as f:
+        with open(os.path.join(ROOT, "profiles", "ced_projection_traffic.json")) as f:
             cap = json.load(f)
         csrc = os.path.join(ROOT, "sparse_attention_decode_kv_b200", "csrc")
         text = "".join(open(os.path.join(csrc, n)).read() for n in ("ced.cu", "tcgen05.cuh", "common.cuh"))
@@ -756,7 +756,7 @@ def run_ced(args, world, rank, local):
                    "d": d, "channels": 512,
                    "l2": "inputs larger than L2 (h is %.0f MB)" % (h.numel() * 2 / 1e6),
                    "parallelism": f"dp{world} (independent token batches)"},
-        "roofline": {"kernel": "ced_quant_kernel (tcgen05 GEMM + MXFP4 epilogue)",
+        "roofline": {"kernel": "ced_pair_kernel (tcgen05 cta_group::2 GEMM + MXFP4 epilogue)",
                      "bound": "tensor", "achieved": round(tflops, 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "peak_kind": peak_kind,
                      "algorithmic_flop_per_launch": flop, "launch_ms": round(ms, 4),
