@@ -174,7 +174,7 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return p;
 }
 
-// 3-D tiled bulk tensor load into this CTA's shared memory, completing on `bar` (no multicast).
+// 3-D tiled bulk tensor load into this CTA's shared memory, completing on `bar` (this CTA only).
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y, int z, uint64_t policy) {
   asm volatile(

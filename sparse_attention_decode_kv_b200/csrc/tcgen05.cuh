@@ -101,7 +101,7 @@ __device__ __forceinline__ void tmem_wait_ld() {
 
 // ----------------------------------------------------------------------------------------- TMA
 
-// 2-D tiled bulk tensor load into this CTA's shared memory, completing on `bar` (no multicast).
+// 2-D tiled bulk tensor load into this CTA's shared memory, completing on `bar` (this CTA only).
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
                                             int y) {
   asm volatile(
