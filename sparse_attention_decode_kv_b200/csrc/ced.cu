@@ -62,9 +62,8 @@ constexpr int kCedEpiWarps = 4;
 constexpr int kCedATile = kCedM * kCedK * 2;  // 16 KiB
 constexpr int kCedBTile = kCedN * kCedK * 2;  // 32 KiB
 constexpr int kCedTmemCols = 2 * kCedN;       // two accumulators: the whole tensor memory
-constexpr int kCedNHalf = kCedN / 2;           // width of the tail tiles (see ProjArgs::split_from)
+constexpr int kCedNHalf = kCedN / 2;           // channels of a tile one CTA of a pair loads
 constexpr uint32_t kCedIdesc = umma_idesc_bf16_f32(kCedM, kCedN);
-constexpr uint32_t kCedIdescHalf = umma_idesc_bf16_f32(kCedM, kCedNHalf);
 
 static_assert(kCedN * (D / kCedN) == D, "two channel tiles cover the 512 latent channels");
 
@@ -124,10 +123,6 @@ struct ProjArgs {
   int n;       // rows per sequence (kEpiMxfp4Cache: token i of sequence b is row b n + i)
   int d;       // reduction length, a multiple of kCedK
   int ksplit;  // tile groups the d-slices are split over (1 for kEpiMxfp4Cache), <= d / kCedK
-  // Tiles from split_from on are the last partial wave of the full-width tiles, each cut into two
-  // 128-channel halves, so that wave takes about half as long (tiles total = split_from +
-  // 2 * (full-width tiles - split_from)). split_from = the tile count disables it.
-  int split_from;
   const int32_t* pos;
   int n_cap;
   uint8_t* codes;
@@ -136,24 +131,13 @@ struct ProjArgs {
   int32_t* dev_err;
 };
 
-// Full-width tile t: channel half t % 2; then (t / 2) = token tile * ksplit + d-split. From
-// split_from on, tile split_from + 2 u + h is the half h of full-width tile split_from + u.
+// Tile t: channel half t % 2; then (t / 2) = token tile * ksplit + d-split.
 struct ProjTile {
-  int m0, n0, nw, kb, ke, ks;
+  int m0, n0, kb, ke, ks;
 };
-__device__ __forceinline__ ProjTile proj_tile(int t, int ksplit, int nk, int split_from) {
+__device__ __forceinline__ ProjTile proj_tile(int t, int ksplit, int nk) {
   ProjTile r;
-  int sub = -1;
-  if (t >= split_from) {
-    sub = (t - split_from) & 1;
-    t = split_from + ((t - split_from) >> 1);
-  }
   r.n0 = (t & 1) * kCedN;
-  r.nw = kCedN;
-  if (sub >= 0) {
-    r.n0 += sub * kCedNHalf;
-    r.nw = kCedNHalf;
-  }
   const int u = t >> 1;
   const int mt = u / ksplit;
   r.ks = u - mt * ksplit;
@@ -165,16 +149,14 @@ __device__ __forceinline__ ProjTile proj_tile(int t, int ksplit, int nk, int spl
 
 template <int kEpi>
 __device__ __forceinline__ void proj_body(const CUtensorMap* tm_h, const CUtensorMap* tm_w,
-                                          const CUtensorMap* tm_w_half, const ProjArgs& a) {
+                                          const ProjArgs& a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   CedSmem& sm = *reinterpret_cast<CedSmem*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int M = a.M, n = a.n, ksplit = a.ksplit;
   const int nk = a.d / kCedK;
   int32_t* dev_err = a.dev_err;
-  const int split_from = a.split_from;
-  const int full_tiles = ((M + kCedM - 1) / kCedM) * (D / kCedN) * ksplit;
-  const int tiles = split_from + 2 * (full_tiles - split_from);
+  const int tiles = ((M + kCedM - 1) / kCedM) * (D / kCedN) * ksplit;
   const int my_tiles = tiles > static_cast<int>(blockIdx.x)
                            ? (tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
                            : 0;
@@ -209,8 +191,7 @@ __device__ __forceinline__ void proj_body(const CUtensorMap* tm_h, const CUtenso
       int it = 0;  // stage uses so far (the ring runs on across tiles)
       for (int j = 0; j < my_tiles && !*abort; ++j) {
         const int t = static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x);
-        const ProjTile pt = proj_tile(t, ksplit, nk, split_from);
-        const bool half = pt.nw != kCedN;
+        const ProjTile pt = proj_tile(t, ksplit, nk);
         for (int kc = pt.kb; kc < pt.ke; ++kc, ++it) {
           const int s = it % kCedStages;
           if (it >= kCedStages &&
@@ -219,9 +200,9 @@ __device__ __forceinline__ void proj_body(const CUtensorMap* tm_h, const CUtenso
             *abort = 1;
             break;
           }
-          mbar_arrive_expect_tx(&sm.full[s], kCedATile + (half ? kCedBTile / 2 : kCedBTile));
+          mbar_arrive_expect_tx(&sm.full[s], kCedATile + kCedBTile);
           tma_load_2d(sm.a[s], tm_h, &sm.full[s], kc * kCedK, pt.m0);
-          tma_load_2d(sm.b[s], half ? tm_w_half : tm_w, &sm.full[s], kc * kCedK, pt.n0);
+          tma_load_2d(sm.b[s], tm_w, &sm.full[s], kc * kCedK, pt.n0);
         }
       }
       // drain: every issued copy must land before the CTA may exit
@@ -244,8 +225,7 @@ __device__ __forceinline__ void proj_body(const CUtensorMap* tm_h, const CUtenso
         tcgen05_fence_after();
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kCedN);
         const ProjTile pt = proj_tile(static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x),
-                                      ksplit, nk, split_from);
-        const uint32_t idesc = pt.nw == kCedN ? kCedIdesc : kCedIdescHalf;
+                                      ksplit, nk);
         bool ok = true;
         for (int kc = pt.kb; kc < pt.ke; ++kc, ++it) {
           const int s = it % kCedStages;
@@ -259,7 +239,7 @@ __device__ __forceinline__ void proj_body(const CUtensorMap* tm_h, const CUtenso
           const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
 #pragma unroll
           for (int k4 = 0; k4 < kCedK / 16; ++k4)  // 16 bf16 = 32 bytes per instruction
-            umma_bf16(d_tmem, umma_desc_k128(a0 + 32 * k4), umma_desc_k128(b0 + 32 * k4), idesc,
+            umma_bf16(d_tmem, umma_desc_k128(a0 + 32 * k4), umma_desc_k128(b0 + 32 * k4), kCedIdesc,
                       (kc != pt.kb || k4 != 0) ? 1u : 0u);
           umma_commit(&sm.empty[s]);  // the stage is free once these MMAs have read it
         }
@@ -273,7 +253,7 @@ __device__ __forceinline__ void proj_body(const CUtensorMap* tm_h, const CUtenso
     for (int j = 0; j < my_tiles; ++j) {
       const int acc = j & 1;
       const int t = static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x);
-      const ProjTile pt = proj_tile(t, ksplit, nk, split_from);
+      const ProjTile pt = proj_tile(t, ksplit, nk);
       const int m0 = pt.m0, n0 = pt.n0;
       const bool ok = __all_sync(0xFFFFFFFFu,
                                  bounded_wait(&sm.acc_full[acc], static_cast<uint32_t>((j >> 1) & 1), abort));
@@ -288,7 +268,7 @@ __device__ __forceinline__ void proj_body(const CUtensorMap* tm_h, const CUtenso
       if constexpr (kEpi == kEpiF32Partial) {
         float* prow = a.part + (static_cast<int64_t>(pt.ks) * M + row) * D + n0;
 #pragma unroll 1
-        for (int g = 0; g < pt.nw / 16; ++g) {
+        for (int g = 0; g < kCedN / 16; ++g) {
           uint32_t r[16];
           tmem_ld16(tbase + static_cast<uint32_t>(16 * g), r);
           tmem_wait_ld();
@@ -317,9 +297,8 @@ __device__ __forceinline__ void proj_body(const CUtensorMap* tm_h, const CUtenso
         else if (n0 == 0) flag_error(dev_err, CSA2_DEVERR_POS_RANGE);
       }
       uint32_t sc[16];
-      const int groups = pt.nw / 16;
 #pragma unroll 1
-      for (int g = 0; g < groups; ++g) {
+      for (int g = 0; g < kCedN / 16; ++g) {
         uint32_t r[16];
         tmem_ld16(tbase + static_cast<uint32_t>(16 * g), r);
         tmem_wait_ld();
@@ -337,15 +316,12 @@ __device__ __forceinline__ void proj_body(const CUtensorMap* tm_h, const CUtenso
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.acc_empty[acc]);
       if (dst >= 0) {
-        const uint32_t p0 = sc[0] | (sc[1] << 8) | (sc[2] << 16) | (sc[3] << 24);
-        const uint32_t p1 = sc[4] | (sc[5] << 8) | (sc[6] << 16) | (sc[7] << 24);
-        if (groups == 16) {
-          const uint32_t p2 = sc[8] | (sc[9] << 8) | (sc[10] << 16) | (sc[11] << 24);
-          const uint32_t p3 = sc[12] | (sc[13] << 8) | (sc[14] << 16) | (sc[15] << 24);
-          *reinterpret_cast<uint4*>(scales + dst * (D / 16) + n0 / 16) = make_uint4(p0, p1, p2, p3);
-        } else {  // a 128-channel tail tile: 8 scale bytes
-          *reinterpret_cast<uint2*>(scales + dst * (D / 16) + n0 / 16) = make_uint2(p0, p1);
-        }
+        uint4 packed;
+        packed.x = sc[0] | (sc[1] << 8) | (sc[2] << 16) | (sc[3] << 24);
+        packed.y = sc[4] | (sc[5] << 8) | (sc[6] << 16) | (sc[7] << 24);
+        packed.z = sc[8] | (sc[9] << 8) | (sc[10] << 16) | (sc[11] << 24);
+        packed.w = sc[12] | (sc[13] << 8) | (sc[14] << 16) | (sc[15] << 24);
+        *reinterpret_cast<uint4*>(scales + dst * (D / 16) + n0 / 16) = packed;
       }
     }
   }
@@ -366,14 +342,14 @@ __device__ __forceinline__ void proj_body(const CUtensorMap* tm_h, const CUtenso
 
 __global__ void __launch_bounds__(kCedThreads, 1)
     ced_quant_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w,
-                     const __grid_constant__ CUtensorMap tm_w_half, const ProjArgs a) {
-  proj_body<kEpiMxfp4Cache>(&tm_h, &tm_w, &tm_w_half, a);
+                     const ProjArgs a) {
+  proj_body<kEpiMxfp4Cache>(&tm_h, &tm_w, a);
 }
 
 __global__ void __launch_bounds__(kCedThreads, 1)
     replay_proj_kernel(const __grid_constant__ CUtensorMap tm_h,
                        const __grid_constant__ CUtensorMap tm_w, const ProjArgs a) {
-  proj_body<kEpiF32Partial>(&tm_h, &tm_w, &tm_w, a);  // no half-width tiles
+  proj_body<kEpiF32Partial>(&tm_h, &tm_w, a);
 }
 
 // ---------------------------------------------------------------------------- CTA-pair kernel
@@ -660,7 +636,7 @@ std::mutex g_ced_mu;
 std::vector<int> g_ced_ready;  // per device: shared-memory attributes set
 
 // Tensor maps of h [M, d] (boxes of 128 rows) and w [512, d] (boxes of 256 rows, and of 128
-// rows for the half-width tail tiles when map_w_half is given), 64-wide d-slices with 128-byte
+// rows, one CTA's share of a pair tile, when map_w_half is given), 64-wide d-slices with 128-byte
 // swizzle.
 cudaError_t proj_tensor_maps(const void* h, const void* w, int64_t M, int d, CUtensorMap* map_h,
                              CUtensorMap* map_w, CUtensorMap* map_w_half = nullptr) {
@@ -748,27 +724,21 @@ cudaError_t launch_ced_quant(const void* h, const void* w, int B, int n, int d, 
     count_launches(1);
     return e != cudaSuccess ? e : cudaGetLastError();
   }
-  // A last wave that would fill at most half of the CTAs is cut into half-width tiles, which
-  // then fill at most all of them and finish in about half the time.
+  // fewer than 256 tokens: single CTAs on 128-token tiles
   const int64_t tiles = ((M + kCedM - 1) / kCedM) * (D / kCedN);
-  const int64_t G = std::min<int64_t>(tiles, device_sm_count());
-  const int64_t rem = tiles % G;
-  const int64_t split_from = (rem > 0 && 2 * rem <= G) ? tiles - rem : tiles;
   ProjArgs a{};
   a.M = static_cast<int>(M);
   a.n = n;
   a.d = d;
   a.ksplit = 1;
-  a.split_from = static_cast<int>(split_from);
   a.pos = pos;
   a.n_cap = n_cap;
   a.codes = codes;
   a.scales = scales;
   a.dev_err = dev_err;
-  const dim3 grid(static_cast<unsigned>(G));
+  const dim3 grid(static_cast<unsigned>(std::min<int64_t>(tiles, device_sm_count())));
   profile_begin(CSA2_KERNEL_CED, s);
-  e = launch_pdl(ced_quant_kernel, grid, dim3(kCedThreads), sizeof(CedSmem), s, map_h, map_w,
-                 map_w_half, a);
+  e = launch_pdl(ced_quant_kernel, grid, dim3(kCedThreads), sizeof(CedSmem), s, map_h, map_w, a);
   profile_end(CSA2_KERNEL_CED, s);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
@@ -793,7 +763,6 @@ cudaError_t launch_swa_replay(const void* h, const void* w, int B, int Wr, int d
   a.n = Wr;
   a.d = d;
   a.ksplit = ksplit;
-  a.split_from = static_cast<int>(((M + kCedM - 1) / kCedM) * (D / kCedN) * ksplit);
   a.part = static_cast<float*>(ws);
   a.dev_err = dev_err;
   const int64_t tiles = ((M + kCedM - 1) / kCedM) * (D / kCedN) * ksplit;
