@@ -53,12 +53,13 @@ def _nibbles(codes):
 
 
 @pytest.mark.parametrize("B,n,d", [(2, 200, 256), (1, 128, 64), (3, 77, 4160), (1, 513, 1024),
-                                   (4, 5000, 128), (2, 9500, 64)])
+                                   (4, 5000, 128), (2, 9500, 64), (2, 150, 4160)])
 def test_integer_inputs_bit_exact(gpu, B, n, d):
     """Ragged token tiles, one d-slice (64), a d that wraps the stage ring (4160 = 65 slices).
     Calls of fewer than 256 token rows run on single CTAs; (3, 77, 4160) and (1, 128, 64) take
-    that path. The others run on CTA pairs. With 158 and 150 pair tiles over 74 clusters, each
-    cluster reuses both TMEM accumulators and the last wave is partial."""
+    that path. The others run on CTA pairs; (2, 150, 4160) wraps the pairs' 6-stage ring. With
+    158 and 150 pair tiles over 74 clusters, each cluster reuses both TMEM accumulators and the
+    last wave is partial."""
     rng = np.random.default_rng(B * 7 + n + d)
     h = torch.from_numpy(rng.integers(-3, 4, (B, n, d)).astype(np.float32)).to(torch.bfloat16)
     w = torch.from_numpy(rng.integers(-2, 3, (512, d)).astype(np.float32) / 4).to(torch.bfloat16)
