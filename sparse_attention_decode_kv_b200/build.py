@@ -11,7 +11,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libcsa2.so")
 SOURCES = ["abi.cu", "append.cu", "attend.cu", "ced.cu", "index.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "internal.h", "select.cuh", "tcgen05.cuh"]
+HEADERS = ["common.cuh", "internal.h", "select.cuh", "swa_codec.cuh", "tcgen05.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
