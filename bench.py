@@ -115,20 +115,26 @@ def scan_traffic_per_launch(wl):
         return None
 
 
-def ced_traffic_per_launch(tokens):
-    """DRAM bytes per CED launch from the committed ncu capture (profiles/ced_projection_traffic.json),
-    scaled by token rows; None once the kernel's sources differ from the captured ones."""
+def captured_traffic(record: str):
+    """DRAM bytes per launch from a committed ncu capture (profiles/<record>), or None once the
+    sources the record's hash covers differ from the captured ones."""
     import hashlib
     try:
-        with open(os.path.join(ROOT, "profiles", "ced_projection_traffic.json")) as f:
+        with open(os.path.join(ROOT, "profiles", record)) as f:
             cap = json.load(f)
         csrc = os.path.join(ROOT, "sparse_attention_decode_kv_b200", "csrc")
-        text = "".join(open(os.path.join(csrc, n)).read() for n in ("ced.cu", "tcgen05.cuh", "common.cuh"))
+        text = "".join(open(os.path.join(csrc, n)).read() for n in cap["hash_files"])
         if hashlib.sha256(text.encode()).hexdigest() != cap["source_sha256"]:
             return None
-        return int(round(cap["dram_bytes_per_token"] * tokens))
+        return cap
     except Exception:
         return None
+
+
+def ced_traffic_per_launch(tokens):
+    """CED DRAM bytes per launch (profiles/ced_projection_traffic.json), scaled by token rows."""
+    cap = captured_traffic("ced_projection_traffic.json")
+    return None if cap is None else int(round(cap["dram_bytes_per_token"] * tokens))
 
 
 def algorithmic_bytes(wl) -> dict:
@@ -909,7 +915,9 @@ def run_queries(args, world, rank, local):
                      "frac": round(gbs / peak, 4), "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": byts,
                      "algorithmic_bytes_per_query": per_query,
-                     "launch_ms": round(ms, 4), "traffic": None,
+                     "launch_ms": round(ms, 4),
+                     "traffic": (lambda c: None if c is None else c["dram_bytes_per_launch"])(
+                         captured_traffic("attend_queries_traffic.json")),
                      "note": "algorithmic bytes count every query's gathered rows; neighbouring "
                              "queries share window rows, which L2 serves"},
         "gpu_launches": per_step_launches * Ks,
@@ -1085,7 +1093,8 @@ def run_replay(args, world, rank, local):
                      "peak": peak, "unit": "TFLOP/s",
                      "frac": round(flop / (r_ms / 1e3) / 1e12 / peak, 4), "peak_kind": peak_kind,
                      "algorithmic_flop_per_launch": flop, "launch_ms": round(r_ms, 4),
-                     "traffic": None},
+                     "traffic": (lambda c: None if c is None else c["dram_bytes_per_launch"])(
+                         captured_traffic("replay_traffic.json"))},
         "gpu_launches": per_step_launches * K,
         "clocks": clocks.summary(),
     }
