@@ -118,8 +118,9 @@ CSA2_API int csa2_append_quant(const void *x, const void *ik, int B, int n, cons
 /*
  * CED KV projection with the MXFP4 quantisation in the GEMM epilogue: C = h w^T (bf16 inputs,
  * fp32 accumulation on the tcgen05 tensor cores), each 16-channel group of a row of C quantised
- * exactly as csa2_append_quant quantises an appended entry, and the codes and scales written to
- * the cache rows; the bf16 projection output never reaches memory.
+ * with csa2_append_quant's codec applied to the fp32 values (scale = E4M3 RNE of the fp32
+ * quotient amax/6, codes = E2M1 RNE of the fp32 quotients x/scale), and the codes and scales
+ * written to the cache rows; the projection output never reaches memory.
  * Defines: the CED paragraph of section 一 (the decoder layers' global KV is projected from the
  * middle layer's hidden state, C_l = H_{L/2} W^KV_l) with the FP4 KV cache paragraph.
  *   h         bf16 [B, n, d]: hidden states of the n new tokens of each sequence (row-major).
@@ -128,7 +129,8 @@ CSA2_API int csa2_append_quant(const void *x, const void *ik, int B, int n, cons
  *   d         a multiple of CSA2_CED_D_ALIGN (64), at most CSA2_MAX_CED_D.
  *   pos, n_cap, codes, scales: as csa2_append_quant (token i of sequence b goes to row pos[b]+i).
  * Rows outside [0, n_cap) are skipped with CSA2_DEVERR_POS_RANGE. B * n is at most
- * CSA2_MAX_CED_TOKENS. No workspace; launches one kernel.
+ * CSA2_MAX_CED_TOKENS. No workspace; launches one kernel (clusters of two CTAs sharing each
+ * MMA when B * n >= 256, single CTAs below).
  */
 enum { CSA2_CED_D_ALIGN = 64, CSA2_MAX_CED_D = 65536, CSA2_MAX_CED_TOKENS = 1 << 26 };
 CSA2_API int csa2_ced_project_quant(const void *h, const void *w, int B, int n, int d,
