@@ -503,39 +503,121 @@ def breakdown(st, steps=20):
 
 
 def run_e2e(st, step, K, W, world, dev):
-    """Same metric through the public API with host buffers: each step copies its inputs from
-    pinned host memory and reads its outputs back."""
+    """Same metric through the public API with host buffers. Every step copies its inputs from
+    pinned host memory and reads its outputs back. Like a serving loop, the transfers overlap
+    the compute: the inputs of step i+1 go in on one copy stream and the outputs of step i-1
+    come back on another while step i runs. There are two device buffer sets, each with its own
+    captured graphs. The timed region runs from the first input copy to the last read-back."""
     stream = torch.cuda.current_stream(dev)
-    host_in = {name: t.detach().cpu().pin_memory() for name, t in
-               (("q", st.q), ("iq", st.iq), ("w", st.w), ("x_new", st.x_new),
-                ("ik_new", st.ik_new))}
-    host_out = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
-    host_lse = torch.empty(st.lse.shape, dtype=st.lse.dtype).pin_memory()
-    dev_in = {"q": st.q, "iq": st.iq, "w": st.w, "x_new": st.x_new, "ik_new": st.ik_new}
+    names_in = ("q", "iq", "w", "x_new", "ik_new")
+    host_in = {k: getattr(st, k).detach().cpu().pin_memory() for k in names_in}
+    sets = [{k: getattr(st, k) for k in names_in + ("out", "lse")},
+            {k: torch.empty_like(getattr(st, k)) for k in names_in + ("out", "lse")}]
+    host_out = [(torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory(),
+                 torch.empty(st.lse.shape, dtype=st.lse.dtype).pin_memory()) for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = host_out.numel() * 4 + host_lse.numel() * 4
+    d2h = host_out[0][0].numel() * 4 + host_out[0][1].numel() * 4
 
-    def e2e_step():
-        for k, t in host_in.items():
-            dev_in[k].copy_(t, non_blocking=True)
-        step()
-        host_out.copy_(st.out, non_blocking=True)
-        host_lse.copy_(st.lse, non_blocking=True)
+    def use(j):
+        for k, t in sets[j].items():
+            setattr(st, k, t)
 
-    for _ in range(W):
-        e2e_step()
+    # graphs of the second buffer set (the caller's graphs read the first)
+    for k in names_in:
+        sets[1][k].copy_(sets[0][k])
+    use(1)
+    g_app1, g_layers1 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_app1, stream=torch.cuda.Stream(dev)):
+        st.append_new()
+    with torch.cuda.graph(g_layers1, stream=torch.cuda.Stream(dev)):
+        st.layers()
+    use(0)
+    torch.cuda.synchronize()
+
+    def step_set(j):
+        if j == 0:
+            step()
+        else:
+            g_app1.replay()
+            use(1)
+            st.index_full()
+            use(0)
+            g_layers1.replay()
+
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    ev_in, ev_step, ev_d2h = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def h2d_copy(i):
+        j = i & 1
+        with torch.cuda.stream(h2d_s):
+            if i >= 2:
+                h2d_s.wait_event(ev_step[j])  # step i-2 no longer reads this set's inputs
+            for k in names_in:
+                sets[j][k].copy_(host_in[k], non_blocking=True)
+            ev_in[j].record(h2d_s)
+
+    def compute(i):
+        j = i & 1
+        stream.wait_event(ev_in[j])
+        if i >= 2:
+            stream.wait_event(ev_d2h[j])  # step i-2's outputs in this set have been read back
+        step_set(j)
+        ev_step[j].record(stream)
+
+    def d2h_copy(i):
+        j = i & 1
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(ev_step[j])
+            host_out[j][0].copy_(sets[j]["out"], non_blocking=True)
+            host_out[j][1].copy_(sets[j]["lse"], non_blocking=True)
+            ev_d2h[j].record(d2h_s)
+
+    def run(n, t0=None, t1=None):
+        if t0 is not None:
+            t0.record(h2d_s)
+        h2d_copy(0)
+        for i in range(n):
+            if i + 1 < n:
+                h2d_copy(i + 1)
+            compute(i)
+            d2h_copy(i)
+        if t1 is not None:
+            t1.record(d2h_s)
+
+    run(max(W, 2))
     torch.cuda.synchronize()
     barrier(world)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(K):
-        e2e_step()
-    t1.record(stream)
+    run(K, t0, t1)
     torch.cuda.synchronize()
     ms = max_over_ranks(world, t0.elapsed_time(t1), dev)
+
+    # the same steps with every copy on the compute stream, one after the other (for contrast)
+    def serial_step():
+        for k in names_in:
+            sets[0][k].copy_(host_in[k], non_blocking=True)
+        step()
+        host_out[0][0].copy_(sets[0]["out"], non_blocking=True)
+        host_out[0][1].copy_(sets[0]["lse"], non_blocking=True)
+
+    torch.cuda.synchronize()
+    barrier(world)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(K):
+        serial_step()
+    s1.record(stream)
+    torch.cuda.synchronize()
+    ms_serial = max_over_ranks(world, s0.elapsed_time(s1), dev)
     return {"value": round(world * st.wl.L * K / (ms / 1e3), 2), "unit": "layer-steps/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "ms_per_step": round(ms / K, 4)}
+            "ms_per_step": round(ms / K, 4),
+            "pipelining": "step i+1's inputs in and step i-1's outputs out on two copy streams "
+                          "while step i runs (two buffer sets, two graph pairs)",
+            "serialized": {"value": round(world * st.wl.L * K / (ms_serial / 1e3), 2),
+                           "ms_per_step": round(ms_serial / K, 4),
+                           "note": "the same copies and steps in order on one stream"}}
 
 
 # --------------------------------------------------------------------------------- oracle arm
