@@ -42,6 +42,10 @@ namespace {
 constexpr int kScanTile = 128;                    // entries per TMA tile
 constexpr int kScanTileBytes = kScanTile * DI * 2;  // 16 KiB
 constexpr int kScanStages = 6;
+// The two consumer groups take alternate tiles, so with an even stage count every stage is always
+// read by the same group and no consumer can be two phases ahead on a stage. With an odd count the
+// groups alternate on a stage, and a parity wait could take a phase two ahead for the one it wants.
+static_assert(kScanStages % 2 == 0, "each ring stage must belong to one consumer group");
 constexpr int kScanGroupWarps = 8;                // warps sharing one tile, 16 entries each
 constexpr int kScanConsumerWarps = 2 * kScanGroupWarps;  // two groups take alternate tiles
 constexpr int kScanThreads = (kScanConsumerWarps + 1) * 32;
