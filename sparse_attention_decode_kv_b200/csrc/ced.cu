@@ -9,6 +9,9 @@
 // quotient x/scale with the sign of x, all codes 0 for a zero scale. Token i of sequence b goes to
 // cache row pos[b] + i.
 //
+// Two kernels project: ced_pair_kernel (further down) for calls of 256 or more token rows, where
+// the two CTAs of a cluster share each MMA, and ced_quant_kernel for smaller calls.
+//
 // ced_quant_kernel: persistent, one CTA per SM; CTA c takes tiles c, c + G, ... of 128 tokens x
 // 256 channels, tile t covering tokens 128 (t / 2) .. and channels 256 (t % 2) .., so the two
 // channel halves of a token tile run at the same time on neighbouring CTAs and the second reads
