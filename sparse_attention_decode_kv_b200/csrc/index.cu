@@ -633,24 +633,26 @@ __global__ void __launch_bounds__(kReThreads)
   }
 }
 
-constexpr int kReCand = 4096;  // reindex candidates at or above the threshold bin
+constexpr int kReRegKeys = 16;  // pool keys per thread in registers (pools of up to 16,384)
 
 struct ReFinalSmem {
-  uint64_t keys[kSmemKeys];
-  uint64_t cand[kReCand];
   int32_t sel[kMaxSel];
+  uint32_t fresh[kDigitBins];  // cleared histogram for the first refining pass
+  uint32_t wc[544];            // per (register slot, warp) counts of the compaction
   SelectScratch sc;
   int nvalid;
   int unsorted;
 };
 
 static_assert(sizeof(ReFinalSmem) <= 227 * 1024, "reindex_final_kernel shared memory");
+static_assert(kFinalThreads == 1024, "the register compaction assumes 1,024 threads");
 
-// One CTA per sequence: the Top-K of the pool's rank keys (0 = empty slot). The key load also
-// histograms the top 12 bits of every real key; only the keys at or above the bin that holds the
-// K-th key enter the radix select (unless more than kReCand do). Winners come out in pool order,
-// which is ascending position for a pool built by the Full-mode indexer; any other pool order is
-// sorted afterwards.
+// One CTA per sequence: the Top-K of the pool's rank keys (0 = empty slot). Pools of up to
+// 16,384 slots are held in registers, 16 keys per thread (slot 1024 j + t in thread t's key j);
+// larger pools are read from global memory on every pass. The key load also histograms the top 12
+// bits of every real key, which fixes those bits of the K-th key; the radix select continues from
+// there over the keys that share them. Winners come out in pool order, which is ascending position
+// for a pool built by the Full-mode indexer; any other pool order is sorted afterwards.
 __global__ void __launch_bounds__(kFinalThreads)
     reindex_final_kernel(const uint64_t* __restrict__ keys_g, int L, int K,
                          int32_t* __restrict__ topk) {
@@ -660,57 +662,79 @@ __global__ void __launch_bounds__(kFinalThreads)
   pdl_launch_dependents();
   const int b = blockIdx.x, tid = threadIdx.x;
   const uint64_t* src = keys_g + static_cast<int64_t>(b) * L;
-  const bool in_smem = L <= kSmemKeys;
-  for (int i = tid; i < kDigitBins; i += kFinalThreads) sm.sc.hist[i] = 0u;
+  const bool in_regs = L <= kReRegKeys * kFinalThreads;
+  for (int i = tid; i < kDigitBins; i += kFinalThreads) {
+    sm.sc.hist[i] = 0u;
+    sm.fresh[i] = 0u;
+  }
   if (tid == 0) {
     sm.nvalid = 0;
     sm.unsorted = 0;
   }
   __syncthreads();
   int nv = 0;
-  for (int base = 0; base < L; base += 8 * kFinalThreads) {
-    uint64_t v[8];
+  uint64_t key[kReRegKeys];
+  if (in_regs) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = base + j * kFinalThreads + tid;
-      v[j] = i < L ? __ldg(src + i) : 0ull;
+    for (int j = 0; j < kReRegKeys; ++j) {
+      const int i = j * kFinalThreads + tid;
+      key[j] = i < L ? __ldg(src + i) : 0ull;
     }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = base + j * kFinalThreads + tid;
-      if (i < L) {
-        if (in_smem) sm.keys[i] = v[j];
+    for (int j = 0; j < kReRegKeys; ++j)
+      if (key[j] != 0ull) {
+        ++nv;
+        atomicAdd(&sm.sc.hist[static_cast<uint32_t>(key[j] >> 52)], 1u);
+      }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kReRegKeys; ++j) key[j] = 0ull;
+    for (int base = 0; base < L; base += 8 * kFinalThreads) {
+      uint64_t v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = base + j * kFinalThreads + tid;
+        v[j] = i < L ? __ldg(src + i) : 0ull;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
         if (v[j] != 0ull) {
           ++nv;
           atomicAdd(&sm.sc.hist[static_cast<uint32_t>(v[j] >> 52)], 1u);
         }
-      }
     }
   }
   nv = __reduce_add_sync(0xFFFFFFFFu, nv);
   if ((tid & 31) == 0) atomicAdd(&sm.nvalid, nv);
   __syncthreads();
   const int k_take = min(K, sm.nvalid);
-  const uint64_t* c = in_smem ? sm.keys : src;
   if (k_take > 0) {
-    const int T0 = block_find_bin4096(sm.sc.hist, static_cast<uint32_t>(k_take), sm.sc.part,
-                                      sm.sc.ints);
-    const uint32_t n_cand = block_ordered_compact(
-        L, [&](int i) { const uint64_t k = c[i]; return k != 0ull && static_cast<int>(k >> 52) >= T0; },
-        [&](int i, uint32_t slot) { if (slot < kReCand) sm.cand[slot] = c[i]; }, sm.sc.scan);
-    __syncthreads();
-    const bool small = n_cand <= static_cast<uint32_t>(kReCand);
-    const uint64_t* kk = small ? sm.cand : c;
-    const int nk = small ? static_cast<int>(n_cand) : L;
-    auto get = [kk](int i) { return kk[i]; };
-    block_radix_select(get, nk, static_cast<uint32_t>(k_take), sm.sc);
-    const RadixState st = sm.sc.st;
-    block_ordered_compact(
-        nk, [&](int i) { const uint64_t k = kk[i]; return k != 0ull && radix_selected(k, st); },
-        [&](int i, uint32_t slot) {
-          if (slot < kMaxSel) sm.sel[slot] = static_cast<int32_t>(rank_key_index(kk[i]));
-        },
-        sm.sc.scan);
+    radix_state_from_top12(sm.sc.hist, static_cast<uint32_t>(k_take), sm.sc);
+    if (in_regs) {
+      block_radix_refine_visit(
+          [&](auto f) {
+#pragma unroll
+            for (int j = 0; j < kReRegKeys; ++j) f(key[j]);
+          },
+          sm.fresh, sm.sc);
+      const RadixState st = sm.sc.st;
+      block_ordered_compact_regs16(
+          [&](int j) { return key[j] != 0ull && radix_selected(key[j], st); },
+          [&](int j, uint32_t slot) {
+            if (slot < kMaxSel) sm.sel[slot] = static_cast<int32_t>(rank_key_index(key[j]));
+          },
+          sm.wc);
+    } else {
+      auto get = [src](int i) { return __ldg(src + i); };
+      block_radix_refine(get, L, sm.fresh, sm.sc);
+      const RadixState st = sm.sc.st;
+      block_ordered_compact(
+          L, [&](int i) { const uint64_t k = get(i); return k != 0ull && radix_selected(k, st); },
+          [&](int i, uint32_t slot) {
+            if (slot < kMaxSel) sm.sel[slot] = static_cast<int32_t>(rank_key_index(get(i)));
+          },
+          sm.sc.scan);
+    }
     __syncthreads();
     for (int i = tid; i + 1 < k_take; i += kFinalThreads)
       if (sm.sel[i] >= sm.sel[i + 1]) sm.unsorted = 1;

@@ -56,8 +56,9 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
 
 // The largest bin T of a 4096-bin histogram with sum_{bins >= T} >= need (whole CTA; blockDim.x
 // is 256 or 1024, so each thread owns 16 or 4 consecutive bins). `hist` may live in global or
-// shared memory. Three parallel levels: warp sums, then the crossing warp's thread sums, then the
-// crossing thread's bins (kept in registers). part: >= 32 shared words; shared_int: 6 words;
+// shared memory. Each warp publishes its total; after one barrier every warp finds the crossing
+// warp from the 32 totals on its own, and that warp finds the crossing thread and bin (kept in
+// registers), so the search costs two barriers. part: >= 32 shared words; shared_int: 4 words;
 // shared_int[3] receives the count in the bins above T.
 __device__ __forceinline__ int block_find_bin4096(const uint32_t* hist, uint32_t need,
                                                   uint32_t* part, int* shared_int) {
@@ -70,39 +71,30 @@ __device__ __forceinline__ int block_find_bin4096(const uint32_t* hist, uint32_t
   uint32_t s = 0;
 #pragma unroll
   for (int i = 0; i < 16; ++i) s += h[i];
-  const uint32_t wsum = __reduce_add_sync(0xFFFFFFFFu, s);
-  if (lane == 0) part[warp] = wsum;
-  __syncthreads();
-  if (warp == 0) {
-    const uint32_t v = lane < nw ? part[lane] : 0u;
-    uint32_t suf = v;
+  uint32_t suf = s;  // this warp's bins owned by lanes >= lane
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, suf, off);
-      if (lane + off < 32) suf += y;
-    }
-    const uint32_t ball = __ballot_sync(0xFFFFFFFFu, lane < nw && suf >= need);
-    const int wl = ball ? 31 - __clz(ball) : 0;
-    const uint32_t above = __shfl_sync(0xFFFFFFFFu, suf - v, wl);
-    if (lane == 0) {
-      shared_int[0] = wl;
-      shared_int[1] = static_cast<int>(above);
-    }
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, suf, off);
+    if (lane + off < 32) suf += y;
   }
+  if (lane == 0) part[warp] = suf;
   __syncthreads();
-  if (warp == shared_int[0]) {
-    const uint32_t run = static_cast<uint32_t>(shared_int[1]);
-    uint32_t suf = s;
+  // every warp: the crossing warp wl and the count in the warps above it
+  const uint32_t v = lane < nw ? part[lane] : 0u;
+  uint32_t sufw = v;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, suf, off);
-      if (lane + off < 32) suf += y;
-    }
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, sufw, off);
+    if (lane + off < 32) sufw += y;
+  }
+  const uint32_t ballw = __ballot_sync(0xFFFFFFFFu, lane < nw && sufw >= need);
+  const int wl = ballw ? 31 - __clz(ballw) : 0;
+  const uint32_t run = __shfl_sync(0xFFFFFFFFu, sufw - v, wl);
+  if (warp == wl) {
     const uint32_t ball = __ballot_sync(0xFFFFFFFFu, run + suf >= need);
     const int jl = ball ? 31 - __clz(ball) : 0;
-    const uint32_t above = __shfl_sync(0xFFFFFFFFu, suf - s, jl);
     if (lane == jl) {
-      uint32_t r = run + above;
+      uint32_t r = run + suf - s;
       int bin = tid * per;
 #pragma unroll
       for (int i = 15; i >= 0; --i) {
@@ -215,6 +207,76 @@ __device__ void block_radix_select(const Get& get, int n, uint32_t k, SelectScra
   }
 }
 
+// Continues the radix select from sc.st when a first-level histogram of the top 12 key bits has
+// already fixed them (bits = 12, need = what the bin of the k-th key still has to give), so no
+// min/max pass runs. visit(f) calls f(key) for every key the calling thread holds; key 0 marks an
+// empty item and is never counted. fresh: a 4096-word buffer that the caller cleared before its
+// last barrier, used by the first pass so that it needs no clearing barrier (nullptr: clear
+// sc.hist as every later pass does). Same stopping rule as block_radix_select.
+template <class Visit>
+__device__ void block_radix_refine_visit(const Visit& visit, uint32_t* fresh, SelectScratch& sc) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  bool first = true;
+  while (!sc.st.done) {
+    const int bits = sc.st.bits;  // 12 .. 63 here
+    const uint64_t prefix = sc.st.prefix;
+    const int width = min(kDigitBits, 64 - bits);
+    const int shift = 64 - bits - width;
+    const uint64_t dmask = (1ull << width) - 1ull;
+    const uint64_t top = prefix >> (64 - bits);
+    uint32_t* hist = sc.hist;
+    if (first && fresh != nullptr) {
+      hist = fresh;
+    } else {
+      for (int i = tid; i < kDigitBins; i += nt) sc.hist[i] = 0;
+      __syncthreads();
+    }
+    first = false;
+    visit([&](uint64_t key) {
+      if (key != 0ull && (key >> (64 - bits)) == top)
+        atomicAdd(&hist[static_cast<uint32_t>((key >> shift) & dmask)], 1u);
+    });
+    __syncthreads();
+    const uint32_t need = sc.st.need;
+    const int d = block_find_bin4096(hist, need, sc.part, sc.ints);
+    if (tid == 0) {
+      const uint32_t left = need - static_cast<uint32_t>(sc.ints[3]);
+      sc.st.need = left;
+      sc.st.prefix = prefix | (static_cast<uint64_t>(d) << shift);
+      sc.st.bits = bits + width;
+      sc.st.done = (hist[d] == left) || (bits + width == 64);
+    }
+    __syncthreads();
+  }
+}
+
+// block_radix_refine_visit over n keys read with get(i).
+template <class Get>
+__device__ void block_radix_refine(const Get& get, int n, uint32_t* fresh, SelectScratch& sc) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  block_radix_refine_visit(
+      [&](auto f) {
+        for (int i = tid; i < n; i += nt) f(get(i));
+      },
+      fresh, sc);
+}
+
+// Sets sc.st after a first-level histogram `hist` of the top 12 bits of the nonzero keys (held
+// in sc.hist or elsewhere): the bin T0 of the k-th key is fixed, and the select is done if that
+// bin is taken whole. Whole CTA; 1 <= k <= the histogram's total.
+__device__ __forceinline__ void radix_state_from_top12(const uint32_t* hist, uint32_t k,
+                                                       SelectScratch& sc) {
+  const int T0 = block_find_bin4096(hist, k, sc.part, sc.ints);
+  if (threadIdx.x == 0) {
+    const uint32_t left = k - static_cast<uint32_t>(sc.ints[3]);
+    sc.st.prefix = static_cast<uint64_t>(T0) << (64 - kDigitBits);
+    sc.st.bits = kDigitBits;
+    sc.st.need = left;
+    sc.st.done = hist[T0] == left;
+  }
+  __syncthreads();
+}
+
 __device__ __forceinline__ bool radix_selected(uint64_t key, const RadixState& st) {
   if (st.bits == 0) return true;
   return (key >> (64 - st.bits)) >= (st.prefix >> (64 - st.bits));
@@ -246,6 +308,49 @@ __device__ uint32_t block_ordered_compact(int n, const Pred& pred, const Emit& e
     base += __popc(ball);
   }
   __syncthreads();
+  return total;
+}
+
+// Order-preserving compaction over items held in registers by a CTA of 1,024 threads: thread t
+// holds item 1024 j + t in its slot j (j < 16). emit(j, slot) runs for each item with sel(j),
+// slot counting the selected items in item order. The (slot, warp) counts are published in item
+// order and every warp takes its offsets from them after one barrier. wc: 544 shared words (512
+// counts, one pad word after every 16 so that a lane's 16 reads hit distinct banks). Returns the
+// count; the caller synchronises before emitted data is read by other threads or wc is reused.
+template <class Sel, class Emit>
+__device__ uint32_t block_ordered_compact_regs16(const Sel& sel, const Emit& emit, uint32_t* wc) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t m[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    m[j] = __ballot_sync(0xFFFFFFFFu, sel(j));
+    const int e = 32 * j + warp;  // item order of (slot j, warp)
+    if (lane == 0) wc[e + (e >> 4)] = static_cast<uint32_t>(__popc(m[j]));
+  }
+  __syncthreads();
+  // lane l holds entries 16 l .. 16 l + 15; this warp's entries sit at offset warp & 15 of lanes
+  // 2 j + (warp >> 4)
+  uint32_t lsum = 0, lpre = 0;
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const uint32_t cq = wc[17 * lane + q];
+    lpre += q < (warp & 15) ? cq : 0u;
+    lsum += cq;
+  }
+  uint32_t incl = lsum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+  const uint32_t mine = incl - lsum + lpre;
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t base = __shfl_sync(0xFFFFFFFFu, mine, 2 * j + (warp >> 4));
+    if ((m[j] >> lane) & 1u) emit(j, base + static_cast<uint32_t>(__popc(m[j] & lt)));
+  }
   return total;
 }
 
