@@ -332,10 +332,16 @@ __global__ void __launch_bounds__(kCollectThreads)
   if (threadIdx.x == 0) ccnt[static_cast<int64_t>(b) * nchunks + chunk] = total;
 }
 
+constexpr int kRegKeys = 16;  // keys per thread of the register selections (16,384 per CTA)
+
 struct FinalSmem {
   union {
     uint64_t cand[kSmemKeys];        // block candidates (in block order)
     uint32_t skey[2 * kSmemKeys];    // score keys of the selected blocks' positions
+    struct {
+      uint32_t fresh[kDigitBins];    // cleared histogram for the first refining pass
+      uint32_t wc[544];              // per (register slot, warp) counts of the compaction
+    } r;                             // the register selections (which use neither array above)
   } u;
   int32_t wide[kMaxSel];             // top max(K, P) blocks, ascending
   uint64_t wide_key[kMaxSel];        // their rank keys; later the position candidates
@@ -347,26 +353,10 @@ struct FinalSmem {
 
 static_assert(sizeof(FinalSmem) <= 227 * 1024, "index_final_kernel shared memory");
 
-// Rank key of block candidate i, with the chunked layout resolved by a binary search over the
-// chunk prefix (only used when the candidates do not fit in shared memory).
-struct ChunkedKeys {
-  const uint64_t* base;
-  const int32_t* pre;
-  int nchunks;
-  __device__ uint64_t operator()(int i) const {
-    int lo = 0, hi = nchunks - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (pre[mid] <= i) lo = mid;
-      else hi = mid - 1;
-    }
-    return base[static_cast<int64_t>(lo) * kCollectChunk + (i - pre[lo])];
-  }
-};
-
 __global__ void __launch_bounds__(kFinalThreads)
     index_final_kernel(const float* __restrict__ scores, const int32_t* __restrict__ N, int n_cap,
-                       int K, int P, const uint32_t* __restrict__ ccnt,
+                       int K, int P, const uint32_t* __restrict__ hist_g,
+                       const uint32_t* __restrict__ ccnt,
                        const uint64_t* __restrict__ cand, int32_t* __restrict__ topk,
                        int32_t* __restrict__ pool) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -414,46 +404,55 @@ __global__ void __launch_bounds__(kFinalThreads)
   }
   __syncthreads();
   const int C = sm.v.chunk_pre[nch];
-  const bool in_smem = C <= kSmemKeys;
-  if (in_smem) {
-    // copy chunk regions into one ordered array (independent loads, 8 per round)
-    for (int base = 0; base < C; base += 8 * kFinalThreads) {
-      uint64_t vals[8];
-      int dst[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = base + j * kFinalThreads + tid;
-        dst[j] = -1;
-        if (i < C) {
-          int lo = 0, hi = nch - 1;
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (sm.v.chunk_pre[mid] <= i) lo = mid;
-            else hi = mid - 1;
-          }
-          vals[j] = __ldg(cbase + static_cast<int64_t>(lo) * kCollectChunk + (i - sm.v.chunk_pre[lo]));
-          dst[j] = i;
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (dst[j] >= 0) sm.u.cand[dst[j]] = vals[j];
+  auto cand_at = [&](int i) -> uint64_t {  // candidate i in block order (chunk by binary search)
+    int lo = 0, hi = nch - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sm.v.chunk_pre[mid] <= i) lo = mid;
+      else hi = mid - 1;
     }
-    __syncthreads();
-  }
-  const ChunkedKeys gk{cbase, sm.v.chunk_pre, nch};
-  const uint64_t* sk = sm.u.cand;
-  auto cand_key = [&](int i) -> uint64_t { return in_smem ? sk[i] : gk(i); };
+    return __ldg(cbase + static_cast<int64_t>(lo) * kCollectChunk + (i - sm.v.chunk_pre[lo]));
+  };
 
   // ---- top kw blocks, ascending
-  block_radix_select(cand_key, C, static_cast<uint32_t>(kw), sm.sc);
-  {
+  if (C <= kRegKeys * kFinalThreads) {
+    // Candidate 1024 j + t in thread t's key j. The scan's histogram of every block maximum
+    // fixes the top 12 bits of the kw-th key (the candidates are all blocks at or above that
+    // bin); the radix select goes on over the candidates in that bin.
+    for (int i = tid; i < kDigitBins; i += kFinalThreads) sm.u.r.fresh[i] = 0u;
+    uint64_t key[kRegKeys];
+#pragma unroll
+    for (int j = 0; j < kRegKeys; ++j) {
+      const int i = j * kFinalThreads + tid;
+      key[j] = i < C ? cand_at(i) : 0ull;
+    }
+    radix_state_from_top12(hist_g + static_cast<int64_t>(b) * kHistBins, static_cast<uint32_t>(kw),
+                           sm.sc);
+    block_radix_refine_visit(
+        [&](auto f) {
+#pragma unroll
+          for (int j = 0; j < kRegKeys; ++j) f(key[j]);
+        },
+        sm.u.r.fresh, sm.sc);
+    const RadixState st = sm.sc.st;
+    block_ordered_compact_regs16<false>(
+        [&](int j) { return key[j] != 0ull && radix_selected(key[j], st); },
+        [&](int j, uint32_t slot) {
+          if (slot < kMaxSel) {
+            sm.wide[slot] = static_cast<int32_t>(rank_key_index(key[j]));
+            sm.wide_key[slot] = key[j];
+          }
+        },
+        sm.u.r.wc);
+    __syncthreads();
+  } else {
+    block_radix_select(cand_at, C, static_cast<uint32_t>(kw), sm.sc);
     const RadixState st = sm.sc.st;
     block_ordered_compact(
-        C, [&](int i) { return radix_selected(cand_key(i), st); },
+        C, [&](int i) { return radix_selected(cand_at(i), st); },
         [&](int i, uint32_t slot) {
           if (slot < kMaxSel) {
-            const uint64_t key = cand_key(i);
+            const uint64_t key = cand_at(i);
             sm.wide[slot] = static_cast<int32_t>(rank_key_index(key));
             sm.wide_key[slot] = key;
           }
@@ -485,65 +484,105 @@ __global__ void __launch_bounds__(kFinalThreads)
     }
   }
 
-  // ---- position Top-K over every position of the wide blocks (slot order = ascending
-  // position). The score gather also histograms the top 12 bits of each score key; only the
-  // positions at or above the bin that holds the K-th score enter the radix select.
+  // ---- position Top-K over every position of the wide blocks (item i = position i % 8 of block
+  // wide[i / 8]: ascending positions). The score gather also histograms the top 12 bits of each
+  // rank key, which fixes those bits of the K-th key; the radix select continues from there.
   const int L = kw * S;  // <= 32768
   const float* srow = scores + static_cast<int64_t>(b) * n_cap;
-  for (int i = tid; i < kDigitBins; i += kFinalThreads) sm.sc.hist[i] = 0u;
-  __syncthreads();
-  for (int base = 0; base < L; base += 8 * kFinalThreads) {
-    float vals[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = base + j * kFinalThreads + tid;
-      const int p = i < L ? sm.wide[i / S] * S + (i % S) : nb;
-      vals[j] = p < nb ? __ldg(srow + p) : 0.0f;
+  uint32_t n_sel;
+  if (L <= kRegKeys * kFinalThreads) {
+    // position item 1024 j + t in thread t's key j (0: past N or past the wide blocks)
+    for (int i = tid; i < kDigitBins; i += kFinalThreads) {
+      sm.sc.hist[i] = 0u;
+      sm.u.r.fresh[i] = 0u;
     }
+    __syncthreads();
+    // all score loads first: the high word holds the raw score bits until they land, the low
+    // word the inverted position (never 0 for a real position)
+    uint32_t hi[kRegKeys], lo[kRegKeys];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = base + j * kFinalThreads + tid;
-      if (i < L) {
-        const int p = sm.wide[i / S] * S + (i % S);
-        const uint32_t key = p < nb ? float_key(vals[j]) : 0u;  // 0: below every real key
-        sm.u.skey[i] = key;
-        if (p < nb) atomicAdd(&sm.sc.hist[key >> kHistShift], 1u);
+    for (int j = 0; j < kRegKeys; ++j) {
+      const int i = j * kFinalThreads + tid;
+      const int p = i < L ? sm.wide[i / S] * S + (i % S) : nb;
+      lo[j] = p < nb ? ~static_cast<uint32_t>(p) : 0u;
+      hi[j] = p < nb ? __float_as_uint(__ldg(srow + p)) : 0u;
+    }
+    uint64_t key[kRegKeys];
+#pragma unroll
+    for (int j = 0; j < kRegKeys; ++j) {
+      key[j] = lo[j] != 0u ? rank_key(__uint_as_float(hi[j]), ~lo[j]) : 0ull;
+      if (key[j] != 0ull) atomicAdd(&sm.sc.hist[static_cast<uint32_t>(key[j] >> 52)], 1u);
+    }
+    __syncthreads();
+    radix_state_from_top12(sm.sc.hist, static_cast<uint32_t>(kk), sm.sc);
+    block_radix_refine_visit(
+        [&](auto f) {
+#pragma unroll
+          for (int j = 0; j < kRegKeys; ++j) f(key[j]);
+        },
+        sm.u.r.fresh, sm.sc);
+    const RadixState st = sm.sc.st;
+    n_sel = block_ordered_compact_regs16<false>(
+        [&](int j) { return key[j] != 0ull && radix_selected(key[j], st); },
+        [&](int j, uint32_t slot) {
+          if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(rank_key_index(key[j]));
+        },
+        sm.u.r.wc);
+  } else {
+    for (int i = tid; i < kDigitBins; i += kFinalThreads) sm.sc.hist[i] = 0u;
+    __syncthreads();
+    for (int base = 0; base < L; base += 8 * kFinalThreads) {
+      float vals[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = base + j * kFinalThreads + tid;
+        const int p = i < L ? sm.wide[i / S] * S + (i % S) : nb;
+        vals[j] = p < nb ? __ldg(srow + p) : 0.0f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = base + j * kFinalThreads + tid;
+        if (i < L) {
+          const int p = sm.wide[i / S] * S + (i % S);
+          const uint32_t key = p < nb ? float_key(vals[j]) : 0u;  // 0: below every real key
+          sm.u.skey[i] = key;
+          if (p < nb) atomicAdd(&sm.sc.hist[key >> kHistShift], 1u);
+        }
       }
     }
-  }
-  __syncthreads();
-  auto pos_of = [&](int i) { return static_cast<uint32_t>(sm.wide[i / S] * S + (i % S)); };
-  auto pos_key = [&](int i) -> uint64_t {
-    const uint32_t hk = sm.u.skey[i];
-    return hk == 0u ? 0ull : (static_cast<uint64_t>(hk) << 32) | static_cast<uint64_t>(~pos_of(i));
-  };
-  const int T0 = block_find_bin4096(sm.sc.hist, static_cast<uint32_t>(kk), sm.sc.part, sm.sc.ints);
-  // candidates in slot order into the (now free) wide_key array
-  uint64_t* cbuf = sm.wide_key;
-  const uint32_t n_cand = block_ordered_compact(
-      L, [&](int i) { const uint32_t k = sm.u.skey[i]; return k != 0u && static_cast<int>(k >> kHistShift) >= T0; },
-      [&](int i, uint32_t slot) { if (slot < kMaxSel) cbuf[slot] = pos_key(i); }, sm.sc.scan);
-  __syncthreads();
-  uint32_t n_sel;
-  if (n_cand <= static_cast<uint32_t>(kMaxSel)) {
-    auto get = [cbuf](int i) { return cbuf[i]; };
-    block_radix_select(get, static_cast<int>(n_cand), static_cast<uint32_t>(kk), sm.sc);
-    const RadixState st = sm.sc.st;
-    n_sel = block_ordered_compact(
-        static_cast<int>(n_cand), [&](int i) { return radix_selected(cbuf[i], st); },
-        [&](int i, uint32_t slot) {
-          if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(rank_key_index(cbuf[i]));
-        },
-        sm.sc.scan);
-  } else {
-    block_radix_select(pos_key, L, static_cast<uint32_t>(kk), sm.sc);
-    const RadixState st = sm.sc.st;
-    n_sel = block_ordered_compact(
-        L, [&](int i) { const uint64_t k = pos_key(i); return k != 0ull && radix_selected(k, st); },
-        [&](int i, uint32_t slot) {
-          if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(pos_of(i));
-        },
-        sm.sc.scan);
+    __syncthreads();
+    auto pos_of = [&](int i) { return static_cast<uint32_t>(sm.wide[i / S] * S + (i % S)); };
+    auto pos_key = [&](int i) -> uint64_t {
+      const uint32_t hk = sm.u.skey[i];
+      return hk == 0u ? 0ull : (static_cast<uint64_t>(hk) << 32) | static_cast<uint64_t>(~pos_of(i));
+    };
+    const int T0 = block_find_bin4096(sm.sc.hist, static_cast<uint32_t>(kk), sm.sc.part, sm.sc.ints);
+    // candidates in slot order into the (now free) wide_key array
+    uint64_t* cbuf = sm.wide_key;
+    const uint32_t n_cand = block_ordered_compact(
+        L, [&](int i) { const uint32_t k = sm.u.skey[i]; return k != 0u && static_cast<int>(k >> kHistShift) >= T0; },
+        [&](int i, uint32_t slot) { if (slot < kMaxSel) cbuf[slot] = pos_key(i); }, sm.sc.scan);
+    __syncthreads();
+    if (n_cand <= static_cast<uint32_t>(kMaxSel)) {
+      auto get = [cbuf](int i) { return cbuf[i]; };
+      block_radix_select(get, static_cast<int>(n_cand), static_cast<uint32_t>(kk), sm.sc);
+      const RadixState st = sm.sc.st;
+      n_sel = block_ordered_compact(
+          static_cast<int>(n_cand), [&](int i) { return radix_selected(cbuf[i], st); },
+          [&](int i, uint32_t slot) {
+            if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(rank_key_index(cbuf[i]));
+          },
+          sm.sc.scan);
+    } else {
+      block_radix_select(pos_key, L, static_cast<uint32_t>(kk), sm.sc);
+      const RadixState st = sm.sc.st;
+      n_sel = block_ordered_compact(
+          L, [&](int i) { const uint64_t k = pos_key(i); return k != 0ull && radix_selected(k, st); },
+          [&](int i, uint32_t slot) {
+            if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(pos_of(i));
+          },
+          sm.sc.scan);
+    }
   }
   for (int i = static_cast<int>(n_sel) + tid; i < K; i += kFinalThreads) topk_out[i] = -1;
 }
@@ -718,7 +757,7 @@ __global__ void __launch_bounds__(kFinalThreads)
           },
           sm.fresh, sm.sc);
       const RadixState st = sm.sc.st;
-      block_ordered_compact_regs16(
+      block_ordered_compact_regs16<true>(
           [&](int j) { return key[j] != 0ull && radix_selected(key[j], st); },
           [&](int j, uint32_t slot) {
             if (slot < kMaxSel) sm.sel[slot] = static_cast<int32_t>(rank_key_index(key[j]));
@@ -855,8 +894,8 @@ cudaError_t launch_index_full(const void* iq, const float* w, const void* ik_cac
   if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
   e = launch_pdl(index_final_kernel, dim3(B), dim3(kFinalThreads), sizeof(FinalSmem), s,
                  static_cast<const float*>(scores), N, n_cap, K, P,
-                 static_cast<const uint32_t*>(ccnt), static_cast<const uint64_t*>(cand), topk,
-                 pool);
+                 static_cast<const uint32_t*>(hist), static_cast<const uint32_t*>(ccnt),
+                 static_cast<const uint64_t*>(cand), topk, pool);
   profile_end(CSA2_KERNEL_INDEX_SELECT, s);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();

@@ -277,9 +277,11 @@ __device__ __forceinline__ void radix_state_from_top12(const uint32_t* hist, uin
   __syncthreads();
 }
 
+// Is key among the selected ones, i.e. are its top st.bits bits >= those of the threshold? Every
+// select leaves the bits of st.prefix below its top st.bits at zero (and st.prefix = 0 when
+// st.bits = 0), so comparing the shifted words is the same as comparing the keys themselves.
 __device__ __forceinline__ bool radix_selected(uint64_t key, const RadixState& st) {
-  if (st.bits == 0) return true;
-  return (key >> (64 - st.bits)) >= (st.prefix >> (64 - st.bits));
+  return key >= st.prefix;
 }
 
 // Order-preserving compaction over items 0..n-1 (whole CTA): emit(i, slot) is called for every
@@ -317,15 +319,18 @@ __device__ uint32_t block_ordered_compact(int n, const Pred& pred, const Emit& e
 // order and every warp takes its offsets from them after one barrier. wc: 544 shared words (512
 // counts, one pad word after every 16 so that a lane's 16 reads hit distinct banks). Returns the
 // count; the caller synchronises before emitted data is read by other threads or wc is reused.
-template <class Sel, class Emit>
+// kKeepMasks: keep the 16 ballot masks in registers across the barrier, or form them again after
+// it (for callers short of registers).
+template <bool kKeepMasks, class Sel, class Emit>
 __device__ uint32_t block_ordered_compact_regs16(const Sel& sel, const Emit& emit, uint32_t* wc) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t m[16];
+  uint32_t mk[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    m[j] = __ballot_sync(0xFFFFFFFFu, sel(j));
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, sel(j));
+    if (kKeepMasks) mk[j] = m;
     const int e = 32 * j + warp;  // item order of (slot j, warp)
-    if (lane == 0) wc[e + (e >> 4)] = static_cast<uint32_t>(__popc(m[j]));
+    if (lane == 0) wc[e + (e >> 4)] = static_cast<uint32_t>(__popc(m));
   }
   __syncthreads();
   // lane l holds entries 16 l .. 16 l + 15; this warp's entries sit at offset warp & 15 of lanes
@@ -349,7 +354,8 @@ __device__ uint32_t block_ordered_compact_regs16(const Sel& sel, const Emit& emi
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const uint32_t base = __shfl_sync(0xFFFFFFFFu, mine, 2 * j + (warp >> 4));
-    if ((m[j] >> lane) & 1u) emit(j, base + static_cast<uint32_t>(__popc(m[j] & lt)));
+    const uint32_t m = kKeepMasks ? mk[j] : __ballot_sync(0xFFFFFFFFu, sel(j));
+    if ((m >> lane) & 1u) emit(j, base + static_cast<uint32_t>(__popc(m & lt)));
   }
   return total;
 }
