@@ -41,9 +41,11 @@
  *   - Kernels after the first of a call are launched with programmatic dependent launch: each may
  *     start while the kernel before it on the stream finishes, and waits for it before reading
  *     anything a kernel can have produced. Kernels outside this library never trigger that early
- *     start, so their results are complete before a call begins. The attention kernels read q
- *     before the wait, since no kernel of this library writes q: q must not alias memory that the
- *     preceding calls of this library on the stream write.
+ *     start, so their results are complete before a call begins. The attention kernels read q, N,
+ *     swa_len (and qseq, swa_lo) before the wait, since no kernel of this library writes them:
+ *     they must not alias memory that the preceding calls of this library on the stream write.
+ *     csa2_attend in CSA2_MODE_REUSE also reads idx and the first tile's codes and scales before
+ *     the wait (see there).
  */
 #ifndef CSA2_H
 #define CSA2_H
@@ -247,7 +249,13 @@ CSA2_API int csa2_index_reindex_noalloc(const void *iq, const float *w, const vo
  * Sparse attention over the selected MXFP4 entries and the FP8 SWA rows, all 16 heads.
  * Defines: Reuse mode of section 一 ("sparse attention directly" over reused indices) and the
  * FP8 SWA KV. `mode` records which kind of layer produced idx; it does not change the result
- * (attend(REUSE, idx) == attend(FULL, idx) bit for bit).
+ * (attend(REUSE, idx) == attend(FULL, idx) bit for bit). A Reuse layer's indices, and the cache
+ * rows they name, were produced by an earlier layer, so with CSA2_MODE_REUSE the kernel starts
+ * gathering them before it waits for the preceding kernel on the stream. The caller guarantees
+ * that the immediately preceding call of this library on the stream writes neither idx nor the
+ * codes and scales of the entries idx names. In a decode step that call is the previous layer's
+ * csa2_attend, which writes only out, lse and its workspace. Use CSA2_MODE_FULL or
+ * CSA2_MODE_REINDEX right after the call that produced idx or appended the entries.
  *   q         bf16 [B, 16, 512]; every |q| must be below 65504 (fp16 range).
  *   codes/scales as written by csa2_append_quant; N int32 [B] (device).
  *   idx       int32 [B, K]: entry positions, -1 = none; duplicates count as separate entries.

@@ -236,7 +236,7 @@ int csa2_attend(int mode, const void* q, float softmax_scale, const uint8_t* cod
   return cuda_status(csa2::launch_attend(q, softmax_scale, codes, scales, n_cap, N, idx, K,
                                          W > 0 ? swa : nullptr, W > 0 ? swa_scale : nullptr,
                                          W > 0 ? swa_len : nullptr, W, nullptr, nullptr, W, B, B,
-                                         out, lse, ws, dev_err,
+                                         out, lse, ws, dev_err, mode == CSA2_MODE_REUSE,
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -266,7 +266,7 @@ int csa2_attend_queries(const void* q, float softmax_scale, const uint8_t* codes
                                          W > 0 ? swa : nullptr, W > 0 ? swa_scale : nullptr,
                                          W > 0 ? swa_len : nullptr, W, qseq,
                                          W > 0 ? swa_lo : nullptr, S, B, Q, out, lse, ws, dev_err,
-                                         reinterpret_cast<cudaStream_t>(stream)));
+                                         false, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int csa2_cache_restore(const uint8_t* host_codes, const uint8_t* host_scales, const void* host_ik,

@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                   const int32_t* __restrict__ swa_len, int W, const int32_t* __restrict__ qseq,
                   const int32_t* __restrict__ swa_lo, int S, int nseq, float* __restrict__ out,
                   float* __restrict__ lse, float* __restrict__ part_o,
-                  float* __restrict__ part_ml, int32_t* dev_err) {
+                  float* __restrict__ part_ml, int32_t* dev_err, int early_rows) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   AttendSmem& sm = *reinterpret_cast<AttendSmem*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -160,15 +160,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
 
-  pdl_wait();
-  pdl_launch_dependents();
-
   const int tiles_idx = (K + kTile - 1) / kTile;
   const int tiles_swa = (W + kTile - 1) / kTile;
   const int tiles = tiles_idx + tiles_swa;
   const int t_begin = static_cast<int>(static_cast<int64_t>(split) * tiles / nsplit);
   const int t_end = static_cast<int>(static_cast<int64_t>(split + 1) * tiles / nsplit);
 
+  // qseq, N, swa_len and swa_lo, like q, are inputs no kernel of this library writes: they are
+  // read before the wait too
   int sb = qseq ? __ldg(qseq + b) : b;  // cache sequence of query b
   const bool sb_ok = sb >= 0 && sb < nseq;
   if (!sb_ok) {  // an unknown sequence: the query attends to nothing
@@ -199,9 +198,44 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
 
-  // the first tile's indices (possibly written by the preceding kernel)
+  const int64_t seq_row0 = static_cast<int64_t>(sb) * n_cap;
+  const bool first_mx = t_begin < t_end && t_begin < tiles_idx;
+
+  // Software pipeline over MXFP4 tiles: while a tile is computed, the next one's rows stream
+  // into sm.raw with cp.async (its indices were requested when the tile began), so only the
+  // first tile of a CTA and the SWA tiles wait for their gather.
+  int pos_staged[4] = {-1, -1, -1, -1};  // positions of the tile held in sm.raw
+  bool staged = false;
+  // Reuse mode: the indices and the rows they name come from an earlier layer, so the first
+  // tile's gather starts before the wait on the preceding kernel (L2-only loads and copies).
+  if (early_rows && first_mx) {
+    const int r = tid & 15;
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+      const int item = pass * 16 + (tid >> 4);
+      pos_staged[pass] = item < min(kTile, K - t_begin * kTile)
+                             ? __ldcg(idx + static_cast<int64_t>(b) * K + t_begin * kTile + item)
+                             : -1;
+    }
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+      const int item = pass * 16 + (tid >> 4);
+      const bool valid = pos_staged[pass] >= 0 && pos_staged[pass] < nb;
+      const int64_t row = seq_row0 + (valid ? pos_staged[pass] : 0);
+      uint8_t* rr = sm.raw + item * kRawRow;
+      cp_async16(rr + 16 * r, codes + row * (D / 2) + 16 * r, valid ? 16u : 0u);
+      if (r < 2) cp_async16(rr + D / 2 + 16 * r, scales + row * (D / 16) + 16 * r, valid ? 16u : 0u);
+    }
+    cp_async_commit();
+    staged = true;
+  }
+
+  pdl_wait();
+  pdl_launch_dependents();
+
+  // the first tile's indices otherwise (possibly written by the preceding kernel)
   int pos_first[4] = {-1, -1, -1, -1};
-  if (t_begin < t_end && t_begin < tiles_idx) {
+  if (first_mx && !staged) {
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
       const int item = pass * 16 + (tid >> 4);
@@ -215,13 +249,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
 
   const uint32_t q_base = smem_u32(sm.q), v_base = smem_u32(sm.v), p_base = smem_u32(sm.p);
-  const int64_t seq_row0 = static_cast<int64_t>(sb) * n_cap;
-
-  // Software pipeline over MXFP4 tiles: while a tile is computed, the next one's rows stream
-  // into sm.raw with cp.async (its indices were requested when the tile began), so only the
-  // first tile of a CTA and the SWA tiles wait for their gather.
-  int pos_staged[4] = {-1, -1, -1, -1};  // positions of the tile held in sm.raw
-  bool staged = false;
+  if (staged) {  // the early rows have landed (16 threads share an entry's scales)
+    cp_async_wait_all();
+    __syncthreads();
+  }
   for (int tile = t_begin; tile < t_end; ++tile) {
     const bool is_swa = tile >= tiles_idx;
     const int base = is_swa ? (tile - tiles_idx) * kTile : tile * kTile;
@@ -596,7 +627,7 @@ cudaError_t launch_attend(const void* q, float softmax_scale, const uint8_t* cod
                           int K, const uint8_t* swa, const float* swa_scale,
                           const int32_t* swa_len, int W, const int32_t* qseq,
                           const int32_t* swa_lo, int S, int nseq, int B, float* out, float* lse,
-                          void* ws, int32_t* dev_err, cudaStream_t s) {
+                          void* ws, int32_t* dev_err, bool early_rows, cudaStream_t s) {
   const int splits = attend_split_count(B, K, W);
   float* part_o = nullptr;
   float* part_ml = nullptr;
@@ -619,7 +650,7 @@ cudaError_t launch_attend(const void* q, float softmax_scale, const uint8_t* cod
                              static_cast<const uint16_t*>(q), softmax_scale, codes, scales, n_cap,
                              N, idx, K, swa, swa_scale, swa_len, W, qseq, swa_lo, S, nseq, out,
                              lse, part_o, part_ml,
-                             dev_err);
+                             dev_err, early_rows ? 1 : 0);
   count_launches(1);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e == cudaSuccess && splits > 1) {

@@ -34,7 +34,7 @@ cudaError_t launch_attend(const void* q, float softmax_scale, const uint8_t* cod
                           int K, const uint8_t* swa, const float* swa_scale,
                           const int32_t* swa_len, int W, const int32_t* qseq,
                           const int32_t* swa_lo, int S, int nseq, int B, float* out, float* lse,
-                          void* ws, int32_t* dev_err, cudaStream_t s);
+                          void* ws, int32_t* dev_err, bool early_rows, cudaStream_t s);
 
 // Full-mode indexer.
 size_t index_full_workspace_bytes(int B, int n_cap, int K, int P);
