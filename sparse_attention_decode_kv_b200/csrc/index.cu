@@ -53,7 +53,7 @@ constexpr int kCollectChunk = 8192;              // blocks per collect CTA (and 
 constexpr int kCollectThreads = 256;
 constexpr int kFinalThreads = 1024;
 constexpr int kMaxSel = 4096;                     // >= CSA2_MAX_K, CSA2_MAX_P
-constexpr int kSmemKeys = 16384;                  // candidate keys held in shared memory
+constexpr int kSmemKeys = 16384;                  // 8-byte words of the index_final fallback buffer
 
 static_assert(kScanTileBytes == 16384, "tile size");
 
@@ -336,8 +336,7 @@ constexpr int kRegKeys = 16;  // keys per thread of the register selections (16,
 
 struct FinalSmem {
   union {
-    uint64_t cand[kSmemKeys];        // block candidates (in block order)
-    uint32_t skey[2 * kSmemKeys];    // score keys of the selected blocks' positions
+    uint32_t skey[2 * kSmemKeys];    // position fallback: score keys of the wide blocks' positions
     struct {
       uint32_t fresh[kDigitBins];    // cleared histogram for the first refining pass
       uint32_t wc[544];              // per (register slot, warp) counts of the compaction
@@ -672,8 +671,6 @@ __global__ void __launch_bounds__(kReThreads)
   }
 }
 
-constexpr int kReRegKeys = 16;  // pool keys per thread in registers (pools of up to 16,384)
-
 struct ReFinalSmem {
   int32_t sel[kMaxSel];
   uint32_t fresh[kDigitBins];  // cleared histogram for the first refining pass
@@ -701,7 +698,7 @@ __global__ void __launch_bounds__(kFinalThreads)
   pdl_launch_dependents();
   const int b = blockIdx.x, tid = threadIdx.x;
   const uint64_t* src = keys_g + static_cast<int64_t>(b) * L;
-  const bool in_regs = L <= kReRegKeys * kFinalThreads;
+  const bool in_regs = L <= kRegKeys * kFinalThreads;
   for (int i = tid; i < kDigitBins; i += kFinalThreads) {
     sm.sc.hist[i] = 0u;
     sm.fresh[i] = 0u;
@@ -712,22 +709,22 @@ __global__ void __launch_bounds__(kFinalThreads)
   }
   __syncthreads();
   int nv = 0;
-  uint64_t key[kReRegKeys];
+  uint64_t key[kRegKeys];
   if (in_regs) {
 #pragma unroll
-    for (int j = 0; j < kReRegKeys; ++j) {
+    for (int j = 0; j < kRegKeys; ++j) {
       const int i = j * kFinalThreads + tid;
       key[j] = i < L ? __ldg(src + i) : 0ull;
     }
 #pragma unroll
-    for (int j = 0; j < kReRegKeys; ++j)
+    for (int j = 0; j < kRegKeys; ++j)
       if (key[j] != 0ull) {
         ++nv;
         atomicAdd(&sm.sc.hist[static_cast<uint32_t>(key[j] >> 52)], 1u);
       }
   } else {
 #pragma unroll
-    for (int j = 0; j < kReRegKeys; ++j) key[j] = 0ull;
+    for (int j = 0; j < kRegKeys; ++j) key[j] = 0ull;
     for (int base = 0; base < L; base += 8 * kFinalThreads) {
       uint64_t v[8];
 #pragma unroll
@@ -753,7 +750,7 @@ __global__ void __launch_bounds__(kFinalThreads)
       block_radix_refine_visit(
           [&](auto f) {
 #pragma unroll
-            for (int j = 0; j < kReRegKeys; ++j) f(key[j]);
+            for (int j = 0; j < kRegKeys; ++j) f(key[j]);
           },
           sm.fresh, sm.sc);
       const RadixState st = sm.sc.st;

@@ -4,10 +4,12 @@
 // scores (and a Top-2048 of blocks); ties go to the lower index. Every item carries a 64-bit
 // rank key (monotone score key in the high word, inverted index in the low word), so the Top-K is
 // the set of the k largest keys, which are all distinct. The selection is an MSB-first radix
-// select: one min/max pass finds the bits all keys share, then each pass histograms the next 12
-// bits of the keys that still match the known prefix (4096 shared-memory bins) and stops as soon
-// as the bin holding the k-th key is taken whole. Winners are emitted in item order by an
-// order-preserving compaction, so item order (ascending index) needs no sort.
+// select. Each pass histograms the next 12 bits of the keys that still match the known prefix
+// (4,096 shared-memory bins) and stops as soon as the bin holding the k-th key is taken whole.
+// The known prefix starts either from a min/max pass (the bits all keys share) or from a
+// first-level histogram of the top 12 bits that the caller built while loading the keys.
+// Winners are emitted in item order by an order-preserving compaction, over items in memory or
+// over 16 items per thread held in registers, so item order (ascending index) needs no sort.
 #pragma once
 
 #include "common.cuh"
