@@ -18,11 +18,12 @@
 //   block_collect_kernel  finds the histogram bin holding the max(K, P)-th block and copies the
 //                       rank keys of all blocks in or above it, in block order, into one region
 //                       per 8192-block chunk.
-//   index_final_kernel  one CTA per sequence: radix select of the top max(K, P) blocks over the
-//                       candidates, order-preserving compaction (ascending block ids, no sort),
-//                       the pool (top P blocks), then the position Top-K over the positions of
-//                       those blocks: the score gather histograms 12 key bits and only positions
-//                       at or above the K-th score's bin enter the radix select. Every Top-K
+//   index_final_kernel  one CTA per sequence: the top max(K, P) blocks among the candidates
+//                       (held in registers; the scan's histogram fixes the top 12 key bits, the
+//                       radix select refines them), an order-preserving compaction (ascending
+//                       block ids, no sort), the pool (top P blocks), then the position Top-K
+//                       over the positions of those blocks, selected the same way from the
+//                       gathered scores and a histogram built while gathering them. Every Top-K
 //                       position lies in one of the top max(K, P) blocks: a block ranked above
 //                       the block of a selected position holds its own maximum, which outranks
 //                       that position, so fewer than K blocks outrank it.
