@@ -263,7 +263,10 @@ def attend(mode, q, softmax_scale, codes, scales, N, idx, swa, swa_scale, swa_le
            dev_err=None, stream=None) -> None:
     """Sparse attention. q bf16 [B,16,512]; codes/scales as appended; N int32 [B]; idx int32 [B,K];
     swa uint8 [B,W,512] / swa_scale f32 [B,W] / swa_len int32 [B] (or None); out f32 [B,16,512];
-    lse f32 [B,16] or None; ws uint8 workspace (may be empty when none is needed)."""
+    lse f32 [B,16] or None; ws uint8 workspace (may be empty when none is needed).
+    With MODE_REUSE the kernel gathers idx's first rows before it waits for the preceding kernel:
+    the library call right before it on the stream must write neither idx nor those cache rows
+    (in a decode step it is the previous layer's attend)."""
     B, K = idx.shape
     n_cap = codes.shape[1]
     W = 0 if swa is None else swa.shape[1]
