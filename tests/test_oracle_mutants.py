@@ -50,6 +50,12 @@ MUTANTS = {
     "query/key operands swapped": (
         "dot += (double)bf16_to_f32(iq[h * CSA2O_DI + i]) * (double)bf16_to_f32(k[i]);",
         "dot += (double)bf16_to_f32(iq[i]) * (double)bf16_to_f32(k[h * 0 + i]);"),
+    "score tolerance 256x too loose": ("return ldexp(total, -16);", "return ldexp(total, -8);"),
+    "score tolerance 256x too tight": ("return ldexp(total, -16);", "return ldexp(total, -24);"),
+    "score tolerance drops |w|": ("total += fabs((double)w[h]) * s;", "total += (double)w[h] * s;"),
+    "score tolerance sums signed products": (
+        "s += fabs((double)bf16_to_f32(iq[h * CSA2O_DI + i]) * (double)bf16_to_f32(k[i]));",
+        "s += (double)bf16_to_f32(iq[h * CSA2O_DI + i]) * (double)bf16_to_f32(k[i]);"),
 }
 
 
@@ -67,7 +73,8 @@ def _run(name):
             f.write(src.replace(old, new))
         r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                             "tests/test_oracle_codecs.py", "tests/test_oracle_index_attend.py",
-                            "tests/test_oracle_ced.py", "tests/test_oracle_replay.py"],
+                            "tests/test_oracle_ced.py", "tests/test_oracle_replay.py",
+                            "tests/test_oracle_score_tol.py"],
                            cwd=d, capture_output=True, text=True, timeout=600)
         return name, r.returncode
     finally:
