@@ -12,6 +12,8 @@ algorithmic bytes (indexer keys read + gathered MXFP4 codes and scales + FP8 SWA
   python bench.py --ced [--steps K] [--warmup W]
   python bench.py --replay [--replay-n N] [--steps K] [--warmup W]
   python bench.py --queries [--steps K] [--warmup W]
+  python bench.py --append [--steps K] [--warmup W]
+  python bench.py --sweep [--sweep-batches 1,8,64,256] [--steps K] [--warmup W]
 
 --ced measures the CED KV projection with the MXFP4 epilogue instead (8 x 4,096 new tokens,
 hidden size 4,096: a tensor-core-bound GEMM), reported in TFLOP/s against the measured bf16
@@ -24,10 +26,17 @@ causal window of 128 FP8 SWA rows; reported in queries/s and GB/s of gathered by
 (reported against a plain pinned copy of the same bytes) and the replay of their FP8 SWA rings
 from the last 128 tokens' hidden states (d = 4,096; tcgen05 projection, TFLOP/s).
 
+--append measures the MXFP4 quantize-append of 1,048,576 new bf16 entries (N(0,1), 0.1% of the
+elements x20) into one cache: GB/s over the bf16 rows read plus the codes and scales written.
+--sweep measures Reuse-mode attention over N = 131,072 cached entries at batch 1, 8, 64 and 256
+(512 indices per sequence drawn uniformly without replacement, a 128-row SWA window), one JSON
+line per batch size: GB/s over the gathered MXFP4 entries and SWA rows, every call timed alone
+after an L2 flush.
+
 With --gpus N > 1 run under torchrun: every rank decodes its own batch (data parallel, no
 collective on the data path); the step time is the max over ranks.
---impl reference times the CPU oracle (a plain restatement of the same definitions) on a bounded
-sample of the same workload, on rank 0 only.
+--impl reference times the CPU oracle (a plain restatement of the same definitions) on whole decode
+steps of the same workload (every sequence of the batch, one per host thread), on rank 0 only.
 """
 from __future__ import annotations
 
@@ -61,7 +70,8 @@ DEFAULT = workloads.MILLION.name
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 1000; the reference arm's default is 10)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
@@ -75,6 +85,12 @@ def parse():
                     help="tokens per restored sequence for --replay (default 1,048,576)")
     ap.add_argument("--ced", action="store_true",
                     help="measure the CED KV projection with the MXFP4 epilogue instead")
+    ap.add_argument("--append", action="store_true",
+                    help="measure the 1,048,576-entry MXFP4 quantize-append instead")
+    ap.add_argument("--sweep", action="store_true",
+                    help="measure Reuse-mode attention at the sweep's batch sizes (one line each)")
+    ap.add_argument("--sweep-batches", default="1,8,64,256",
+                    help="batch sizes of --sweep (default 1,8,64,256)")
     ap.add_argument("--breakdown", action="store_true",
                     help="also time each library call of the step (eager, synchronised)")
     return ap.parse_args()
@@ -344,12 +360,17 @@ def run_ours(args, world, rank, local):
     st = Stack(wl, dev)
     stream = torch.cuda.current_stream(dev)
 
-    # warm-up (eager), then capture the parts around the Full index into CUDA graphs; the Full
-    # index call is launched eagerly each step so that its scan kernel gets its own events
+    # warm-up (eager), then capture the whole step into one CUDA graph for the headline loop,
+    # which records no events inside the step. A second pass times the scan kernel on its own
+    # events: the append and the layers after the Full index replay from their own graphs and
+    # the Full index is launched eagerly between them, so that its scan gets an event pair.
     launches0 = csa2.launch_count()
     st.eager_step()
     torch.cuda.synchronize()
     per_step_launches = csa2.launch_count() - launches0
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=torch.cuda.Stream(dev)):
+        st.eager_step()
     g_app, g_layers = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_app, stream=torch.cuda.Stream(dev)):
         st.append_new()
@@ -362,14 +383,15 @@ def run_ours(args, world, rank, local):
                for _ in range(K)]
     L = csa2.lib()
 
-    def step(i=None):
+    def step():
+        g_step.replay()
+
+    def probed_step(i):
         g_app.replay()
-        if i is not None:
-            L.csa2_set_profile_events(1, ctypes.c_void_p(ev_scan[i][0].cuda_event),
-                                      ctypes.c_void_p(ev_scan[i][1].cuda_event))
+        L.csa2_set_profile_events(1, ctypes.c_void_p(ev_scan[i][0].cuda_event),
+                                  ctypes.c_void_p(ev_scan[i][1].cuda_event))
         st.index_full()
-        if i is not None:
-            L.csa2_set_profile_events(1, None, None)
+        L.csa2_set_profile_events(1, None, None)
         g_layers.replay()
 
     for e in ev_scan:  # materialise the event handles
@@ -385,9 +407,14 @@ def run_ours(args, world, rank, local):
         barrier(world)
         torch.cuda.synchronize()
         t0.record(stream)
-        for i in range(K):
-            step(i)
+        for _ in range(K):
+            step()
         t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        # roofline pass: the same steps with the scan bracketed by its own events
+        for i in range(K):
+            probed_step(i)
         torch.cuda.synchronize()
         barrier(world)
     ms_local = t0.elapsed_time(t1)
@@ -408,7 +435,7 @@ def run_ours(args, world, rank, local):
     parts = breakdown(st) if args.breakdown else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, dev, samples=wl.B)
+        cpu = cpu_baseline(wl, dev)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "layer-steps/s", "n_gpus": world,
@@ -416,7 +443,7 @@ def run_ours(args, world, rank, local):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16/fp16-in fp32-acc (mxfp4+fp8 cache)",
         "data": "synthetic",
         "config": {"workload": wl.name, "B_per_gpu": wl.B, "N": wl.N, "layers": ",".join(wl.modes),
-                   "K": wl.K, "P": wl.P, "W": wl.W, "cuda_graph": "append+layers; Full index eager",
+                   "K": wl.K, "P": wl.P, "W": wl.W, "cuda_graph": "whole step (append, Full index, layers) as one graph",
                    "l2": "inputs larger than L2 (indexer keys %.2f GB per step)" % (ab["full"] / 1e9),
                    "parallelism": f"dp{world} (independent sequences)"},
         "achieved_gbs": round(achieved_step_gbs, 1),
@@ -428,6 +455,8 @@ def run_ours(args, world, rank, local):
                      "frac": round(scan_gbs / peak, 4), "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": ab["full"],
                      "launch_ms": round(scan_ms, 4), "traffic": scan_traffic_per_launch(wl),
+                     "timing": "CUDA events around every scan launch in a second pass of K steps "
+                               "(append and layers from graphs, the Full index eager)",
                      "traffic_source": "profiles/index_scan_traffic.json (ncu, scaled by entries)"},
         "gpu_launches": per_step_launches * K,
         "clocks": clocks.summary(),
@@ -526,11 +555,9 @@ def run_e2e(st, step, K, W, world, dev):
     for k in names_in:
         sets[1][k].copy_(sets[0][k])
     use(1)
-    g_app1, g_layers1 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_app1, stream=torch.cuda.Stream(dev)):
-        st.append_new()
-    with torch.cuda.graph(g_layers1, stream=torch.cuda.Stream(dev)):
-        st.layers()
+    g_step1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step1, stream=torch.cuda.Stream(dev)):
+        st.eager_step()
     use(0)
     torch.cuda.synchronize()
 
@@ -538,11 +565,7 @@ def run_e2e(st, step, K, W, world, dev):
         if j == 0:
             step()
         else:
-            g_app1.replay()
-            use(1)
-            st.index_full()
-            use(0)
-            g_layers1.replay()
+            g_step1.replay()
 
     h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev = lambda: torch.cuda.Event()
@@ -614,7 +637,7 @@ def run_e2e(st, step, K, W, world, dev):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms / K, 4),
             "pipelining": "step i+1's inputs in and step i-1's outputs out on two copy streams "
-                          "while step i runs (two buffer sets, two graph pairs)",
+                          "while step i runs (two buffer sets, one step graph each)",
             "serialized": {"value": round(world * st.wl.L * K / (ms_serial / 1e3), 2),
                            "ms_per_step": round(ms_serial / K, 4),
                            "note": "the same copies and steps in order on one stream"}}
@@ -648,97 +671,140 @@ def oracle_rows(wl, b, rows, dev):
     return res
 
 
-def oracle_one_sequence(wl, sample, dev):
-    """Time the oracle on one sequence's full stack step. Returns seconds of oracle compute (data
-    preparation between the index and attention parts is not timed)."""
-    import numpy as np
+def host_threads() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
 
-    import oracle
-    N, K, P, W = wl.N, wl.K, wl.P, wl.W
-    ik = sample["ik"][None]
-    t_index = 0.0
-    topks = []
-    t = time.perf_counter()
-    r = oracle.index_full(sample["iq"][0][None], sample["w"][0][None], ik, [N], K, P)
-    t_index += time.perf_counter() - t
-    pool = r["pool"]
-    topks.append(r["topk"][0])
-    j = 1
-    per_layer = []
-    for m in wl.modes:
-        if m == "F":
-            per_layer.append(topks[0])
-        elif m == "RI":
-            t = time.perf_counter()
-            rr = oracle.index_reindex(sample["iq"][j][None], sample["w"][j][None], ik, pool, K)
-            t_index += time.perf_counter() - t
-            topks.append(rr["topk"][0])
-            per_layer.append(rr["topk"][0])
-            j += 1
-        else:
-            per_layer.append(per_layer[-1])
-    # untimed: the oracle quantises the rows the attention needs (remapped to a compact cache)
-    need = sorted(set(int(v) for tk in per_layer for v in tk if v >= 0))
-    rows = oracle_rows(wl, sample["b"], need, dev)
-    codes, scales = oracle.mxfp4_quantize(rows)
-    remap = {p: i for i, p in enumerate(need)}
-    swa_rows = oracle_rows(wl, sample["b"], list(range(N - min(N, W), N)), dev)
-    swa, swsc = oracle.swa_quantize(swa_rows)
-    # ring slot of position p is p mod W
-    ring = np.zeros((W, 512), np.uint8)
-    rsc = np.zeros((W,), np.float32)
-    for i, p in enumerate(range(N - min(N, W), N)):
-        ring[p % W], rsc[p % W] = swa[i], swsc[i]
-    t_att = 0.0
-    for l, tk in enumerate(per_layer):
-        idx = np.array([remap[int(v)] if v >= 0 else -1 for v in tk], np.int64)
+
+class OracleDecode:
+    """The oracle's decode step (Full index, Reindex layers, every layer's attention) for a set of
+    sequences, one sequence per host thread. The oracle itself is plain single-threaded C; ctypes
+    releases the GIL while it runs, so the sequences proceed in parallel. Between the index part
+    and the attention part the rows the attention needs are regenerated and quantised by the
+    oracle into a compact cache; that preparation is not timed and is kept for later steps."""
+
+    def __init__(self, wl, dev, seqs, threads):
+        import concurrent.futures as cf
+        self.wl, self.dev = wl, dev
+        self.inputs, _ = oracle_sample_inputs(wl, dev, seqs)
+        self.threads = max(1, min(threads, len(self.inputs)))
+        self.pool = cf.ThreadPoolExecutor(max_workers=self.threads)
+        self.prep = {}
+
+    def close(self):
+        self.pool.shutdown()
+
+    def _index(self, sample):
+        import oracle
+        wl = self.wl
+        ik = sample["ik"][None]
+        r = oracle.index_full(sample["iq"][0][None], sample["w"][0][None], ik, [wl.N], wl.K, wl.P)
+        per_layer, j, cur = [], 1, r["topk"][0]
+        for m in wl.modes:
+            if m == "RI":
+                cur = oracle.index_reindex(sample["iq"][j][None], sample["w"][j][None], ik,
+                                           r["pool"], wl.K)["topk"][0]
+                j += 1
+            per_layer.append(cur)
+        return per_layer
+
+    def _prepare(self, sample, per_layer):
+        import numpy as np
+
+        import oracle
+        wl, b = self.wl, sample["b"]
+        key = tuple(tuple(int(v) for v in tk) for tk in per_layer)
+        hit = self.prep.get(b)
+        if hit is not None and hit[0] == key:
+            return hit[1]
+        N, W = wl.N, wl.W
+        need = sorted(set(int(v) for tk in per_layer for v in tk if v >= 0))
+        codes, scales = oracle.mxfp4_quantize(oracle_rows(wl, b, need, self.dev))
+        remap = {p: i for i, p in enumerate(need)}
+        swa, swsc = oracle.swa_quantize(oracle_rows(wl, b, list(range(N - min(N, W), N)), self.dev))
+        ring = np.zeros((W, 512), np.uint8)
+        rsc = np.zeros((W,), np.float32)
+        for i, p in enumerate(range(N - min(N, W), N)):  # ring slot of position p is p mod W
+            ring[p % W], rsc[p % W] = swa[i], swsc[i]
+        idx = [np.array([remap[int(v)] if v >= 0 else -1 for v in tk], np.int64) for tk in per_layer]
+        prep = (codes, scales, idx, ring, rsc)
+        self.prep[b] = (key, prep)
+        return prep
+
+    def _attend(self, sample, prep):
+        import oracle
+        wl = self.wl
+        codes, scales, idx, ring, rsc = prep
+        for l in range(wl.L):
+            oracle.attend_seq(sample["q"][l], wl.softmax_scale, codes, scales, idx[l], ring, rsc,
+                              min(wl.N, wl.W))
+
+    def step(self) -> float:
+        """Seconds of oracle compute for one decode step of every sequence in the set."""
         t = time.perf_counter()
-        oracle.attend_seq(sample["q"][l], wl.softmax_scale, codes, scales, idx, ring, rsc, min(N, W))
-        t_att += time.perf_counter() - t
-    return t_index + t_att
+        per = list(self.pool.map(self._index, self.inputs))
+        t_index = time.perf_counter() - t
+        preps = [self._prepare(smp, p) for smp, p in zip(self.inputs, per)]  # not timed
+        t = time.perf_counter()
+        list(self.pool.map(self._attend, self.inputs, preps))
+        return t_index + time.perf_counter() - t
 
 
-def cpu_baseline(wl, dev, samples=1):
-    seqs = list(range(min(samples, wl.B)))
-    inputs, _ = oracle_sample_inputs(wl, dev, seqs)
-    secs = [oracle_one_sequence(wl, s, dev) for s in inputs]
-    per_seq = statistics.mean(secs)
-    value = wl.L / (per_seq * wl.B)
-    return {"value": round(value, 4), "unit": "layer-steps/s", "cores": 1, "kind": "oracle",
-            "sample": (f"{len(seqs)} of {wl.B} sequences through all {wl.L} layers "
+def cpu_baseline(wl, dev):
+    """One oracle decode step of the whole batch, one sequence per host thread."""
+    od = OracleDecode(wl, dev, list(range(wl.B)), host_threads())
+    try:
+        sec = od.step()
+    finally:
+        od.close()
+    return {"value": round(wl.L / sec, 4), "unit": "layer-steps/s", "cores": od.threads,
+            "kind": "oracle",
+            "sample": (f"one whole decode step: all {wl.B} sequences through all {wl.L} layers "
                        f"(Full index over N={wl.N}, {sum(m == 'RI' for m in wl.modes)} Reindex, "
-                       f"{wl.L} attentions), scaled to the batch: {per_seq:.2f} s per sequence"),
-            "seconds": round(sum(secs), 2)}
+                       f"{wl.L} attentions), one sequence per thread: {sec:.2f} s"),
+            "seconds": round(sec, 2)}
+
+
+REFERENCE_DEFAULT_STEPS = 10
 
 
 def run_reference(args, world, rank, local):
+    """The oracle timed as the reference arm: every step is one whole decode step of the batch
+    (all B sequences, one per host thread), so ms_per_step is the wall time of one step."""
     if rank != 0:
         return
     from oracle import build as oracle_build
     oracle_build.build()
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
     wl = WORKLOADS[args.workload]
-    inputs, _ = oracle_sample_inputs(wl, dev, [0])
-    for _ in range(args.warmup):
-        oracle_one_sequence(wl, inputs[0], dev)
-    secs = [oracle_one_sequence(wl, inputs[0], dev) for _ in range(args.steps)]
-    per_seq = statistics.mean(secs)
-    value = wl.L / (per_seq * wl.B)
-    sample = (f"sequence 0 of {wl.B} through all {wl.L} layers per step, scaled to the batch "
-              f"({per_seq:.2f} s per sequence)")
+    steps = args.steps if args.steps is not None else REFERENCE_DEFAULT_STEPS
+    od = OracleDecode(wl, dev, list(range(wl.B)), host_threads())
+    try:
+        for _ in range(args.warmup):
+            od.step()
+        secs = [od.step() for _ in range(steps)]
+    finally:
+        od.close()
+    per_step = statistics.mean(secs)
+    value = wl.L / per_step
+    sample = (f"every step: all {wl.B} sequences through all {wl.L} layers, one sequence per "
+              f"thread on {od.threads} threads ({per_step:.2f} s per step)")
     line = {"metric": METRIC, "value": round(value, 4), "unit": "layer-steps/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(per_seq * wl.B * 1e3, 2), "higher_is_better": True,
+            "steps": steps, "warmup": args.warmup,
+            "ms_per_step": round(per_step * 1e3, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
             "config": {"workload": wl.name, "B_per_gpu": wl.B, "N": wl.N,
-                       "layers": ",".join(wl.modes), "K": wl.K, "P": wl.P, "W": wl.W},
-            "cpu_baseline": {"value": round(value, 4), "unit": "layer-steps/s", "cores": 1,
-                             "kind": "oracle", "sample": sample},
+                       "layers": ",".join(wl.modes), "K": wl.K, "P": wl.P, "W": wl.W,
+                       "parallelism": f"dp{world} (independent sequences)"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "layer-steps/s",
+                             "cores": od.threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "layer-steps/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
-
 
 
 # ------------------------------------------------------------------ CED projection measurement
@@ -1188,8 +1254,345 @@ def run_replay(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------- throughput sweep: append + Reuse
+
+APPEND_METRIC = ("MXFP4 quantize-append GB/s (bf16 rows read + E2M1 codes and E4M3 scales written), "
+                 "1,048,576 entries, 1 B200")
+SWEEP_METRIC = ("Reuse-mode sparse attention GB/s (gathered MXFP4 entries + FP8 SWA rows), "
+                "N=131,072, 1 B200")
+L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
+
+
+def append_cpu_baseline(x, rows=65536):
+    """The oracle's MXFP4 quantisation of `rows` entries, split over the host threads, scaled to
+    GB/s of the same algorithmic bytes per entry."""
+    import concurrent.futures as cf
+
+    import numpy as np
+
+    import oracle
+    from oracle import build as oracle_build
+    oracle_build.build()
+    xb = x.reshape(-1, 512)[:rows].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    threads = max(1, min(host_threads(), 64))
+    parts = np.array_split(xb, threads)
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        t = time.perf_counter()
+        list(ex.map(oracle.mxfp4_quantize, parts))
+        sec = time.perf_counter() - t
+    per_entry = 512 * 2 + 256 + 32
+    return {"value": round(rows * per_entry / sec / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{rows} of {x.shape[0] * x.shape[1]} entries split over {threads} threads "
+                      f"({sec:.2f} s)",
+            "seconds": round(sec, 2)}
+
+
+def run_append(args, world, rank, local):
+    import sparse_attention_decode_kv_b200 as csa2
+    from sparse_attention_decode_kv_b200 import build as csa2_build
+    if rank == 0:
+        csa2_build.build()
+    barrier(world)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = dataclasses.replace(workloads.APPEND_1M, seed=workloads.APPEND_1M.seed + 1000 * rank)
+    x = workloads.append_rows(wl, dev)  # [1, 1,048,576, 512] bf16: 1.07 GB, larger than L2
+    B, n = wl.B, wl.n
+    codes = torch.empty(B, n, 256, dtype=torch.uint8, device=dev)
+    scales = torch.empty(B, n, 32, dtype=torch.uint8, device=dev)
+    pos = torch.zeros(B, dtype=torch.int32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    L = csa2.lib()
+
+    def step():
+        csa2.append_quant(x, None, pos, codes, scales, None, dev_err=err)
+
+    K, Wu = args.steps, args.warmup
+    launches0 = csa2.launch_count()
+    step()
+    torch.cuda.synchronize()
+    per_step_launches = csa2.launch_count() - launches0
+    for _ in range(Wu):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    for a, b in ev:
+        a.record(stream)
+        b.record(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(K):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        for i in range(K):  # the kernel's own launch times, in a second pass
+            L.csa2_set_profile_events(0, ctypes.c_void_p(ev[i][0].cuda_event),
+                                      ctypes.c_void_p(ev[i][1].cuda_event))
+            step()
+            L.csa2_set_profile_events(0, None, None)
+        torch.cuda.synchronize()
+    if int(err.item()):
+        raise RuntimeError(f"device error flags {int(err.item()):#x} during the benchmark")
+    ms = max_over_ranks(world, t0.elapsed_time(t1), dev) / K
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    per_entry = 512 * 2 + 256 + 32
+    byts = B * n * per_entry
+    peak, peak_kind = measured_peak()
+    gbs = world * byts / (ms / 1e3) / 1e9
+    k_gbs = byts / (launch_ms / 1e3) / 1e9
+    e2e = None
+    if not args.no_e2e:
+        # the rows come from pinned host memory every step; the appended cache stays in HBM for
+        # the decode step that reads it, and the step's result read back is the error word
+        x_h = x.cpu().pin_memory()
+        err_h = torch.empty(1, dtype=torch.int32).pin_memory()
+        ke = max(1, min(K, 10))
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(ke):
+            x.copy_(x_h, non_blocking=True)
+            step()
+            err_h.copy_(err, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(world, a.elapsed_time(b), dev) / ke
+        e2e = {"value": round(world * byts / (e_ms / 1e3) / 1e9, 1), "unit": "GB/s",
+               "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": 4,
+               "ms_per_step": round(e_ms, 4),
+               "note": "bounded by the host link: the 1.07 GB of bf16 rows cross it every step"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = append_cpu_baseline(x)
+    line = {
+        "metric": APPEND_METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": Wu, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, e2m1 codes + e4m3 scales out",
+        "data": "synthetic",
+        "config": {"workload": f"append-1M-B{B}-n{n}", "entries": B * n,
+                   "values": "N(0,1), 0.1% of elements x20",
+                   "l2": "inputs larger than L2 (%.2f GB of bf16 rows per step)" % (x.numel() * 2 / 1e9),
+                   "parallelism": f"dp{world} (independent caches)"},
+        "entries_per_s": round(world * B * n / (ms / 1e3), 1),
+        "roofline": {"kernel": "append_kernel (MXFP4 quantize-append)", "bound": "hbm",
+                     "achieved": round(k_gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(k_gbs / peak, 4), "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": byts,
+                     "algorithmic_bytes_per_entry": per_entry, "launch_ms": round(launch_ms, 4),
+                     "traffic": (lambda c: None if c is None else int(round(c["dram_bytes_per_entry"] * B * n)))(
+                         captured_traffic("append_traffic.json")),
+                     "timing": "CUDA events around every append launch in a second pass"},
+        "gpu_launches": per_step_launches * K,
+        "clocks": clocks.summary(),
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def fill_reuse_cache(csa2, wl, cache, dev):
+    """Append every sequence's N rows through the library (the ring keeps the last W)."""
+    for b0 in range(0, wl.B, 16):
+        b1 = min(wl.B, b0 + 16)
+        for c in range(workloads.n_chunks(wl)):
+            x = torch.stack([workloads.reuse_kv_chunk(wl, b, c, dev) for b in range(b0, b1)])
+            pos = torch.full((b1 - b0,), c * workloads.CHUNK, dtype=torch.int32, device=dev)
+            csa2.append_quant(x, None, pos, cache.codes[b0:b1], cache.scales[b0:b1], None,
+                              cache.swa[b0:b1], cache.swa_scale[b0:b1])
+            del x
+    torch.cuda.synchronize()
+
+
+def sweep_cpu_baseline(wl, q, idx, dev, budget_s=4.0):
+    """The oracle's attention for sampled sequences (their rows regenerated and quantised by the
+    oracle, not timed), one sequence per host thread, repeated to about `budget_s`, scaled to
+    GB/s of the same algorithmic bytes."""
+    import concurrent.futures as cf
+
+    import numpy as np
+
+    import oracle
+    from oracle import build as oracle_build
+    oracle_build.build()
+    N, K, W = wl.N, wl.K, wl.W
+    threads = max(1, min(host_threads(), wl.B, 16))
+    seqs = list(range(threads))
+    qb = workloads.bf16_bits(q[seqs])
+    idx_h = idx[seqs].cpu().numpy()
+    wpos = list(range(N - W, N))
+    prep = []
+    for j, b in enumerate(seqs):
+        rows = np.zeros((K, 512), np.uint16)
+        need = idx_h[j].astype(np.int64)
+        for c in np.unique(need // workloads.CHUNK):
+            m = need // workloads.CHUNK == c
+            x = workloads.reuse_kv_chunk(wl, b, int(c), dev)
+            rows[m] = workloads.bf16_bits(x[torch.as_tensor(need[m] - c * workloads.CHUNK, device=dev)])
+        codes, scales = oracle.mxfp4_quantize(rows)
+        xw = workloads.reuse_kv_chunk(wl, b, (N - 1) // workloads.CHUNK, dev)
+        e, sc = oracle.swa_quantize(workloads.bf16_bits(xw[-W:]))
+        ring = np.zeros((W, 512), np.uint8)
+        rsc = np.zeros(W, np.float32)
+        for i, p in enumerate(wpos):
+            ring[p % W], rsc[p % W] = e[i], sc[i]
+        prep.append((qb[j], codes, scales, np.arange(K, dtype=np.int64), ring, rsc))
+
+    def one(p):
+        oracle.attend_seq(p[0], 1.0, p[1], p[2], p[3], p[4], p[5], W)
+
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        reps, sec = 0, 0.0
+        while sec < budget_s:
+            t = time.perf_counter()
+            list(ex.map(one, prep))
+            sec += time.perf_counter() - t
+            reps += 1
+    per_seq = K * 288 + W * 516
+    return {"value": round(reps * threads * per_seq / sec / 1e9, 5), "unit": "GB/s",
+            "cores": threads, "kind": "oracle",
+            "sample": f"{threads} of {wl.B} sequences, one per thread, {reps} rounds ({sec:.2f} s)",
+            "seconds": round(sec, 2)}
+
+
+def run_sweep(args, world, rank, local):
+    import sparse_attention_decode_kv_b200 as csa2
+    from sparse_attention_decode_kv_b200 import build as csa2_build
+    if rank == 0:
+        csa2_build.build()
+    barrier(world)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    L = csa2.lib()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    batches = [int(v) for v in args.sweep_batches.split(",")]
+    for B in batches:
+        base = next((w for w in workloads.REUSE_SWEEP if w.B == B), None)
+        if base is None:
+            base = workloads.ReuseAttendWorkload(f"reuse-attend-B{B}-N131072", B=B)
+        wl = dataclasses.replace(base, seed=base.seed + 1000 * rank)
+        N, K, W = wl.N, wl.K, wl.W
+        cache = csa2.Cache(B, N, W, device=dev)
+        fill_reuse_cache(csa2, wl, cache, dev)
+        idx = workloads.reuse_indices(wl, dev)
+        q = workloads.reuse_queries(wl, dev)
+        out = torch.empty(B, 16, 512, device=dev)
+        lse = torch.empty(B, 16, device=dev)
+        ws = csa2.workspace(csa2.attend_workspace_bytes(B, K, W), dev)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        Nt = torch.full((B,), N, dtype=torch.int32, device=dev)
+        swa_len = torch.full((B,), W, dtype=torch.int32, device=dev)
+
+        def call():
+            csa2.attend(csa2.MODE_REUSE, q, 1.0, cache.codes, cache.scales, Nt, idx, cache.swa,
+                        cache.swa_scale, swa_len, out, lse, ws, err)
+
+        Ks, Wu = args.steps, args.warmup
+        launches0 = csa2.launch_count()
+        call()
+        torch.cuda.synchronize()
+        per_call_launches = csa2.launch_count() - launches0
+        for _ in range(Wu):
+            flush.fill_(1)
+            call()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(Ks)]
+        for a, b in ev:
+            a.record(stream)
+            b.record(stream)
+        # every call follows an L2 flush (a 256 MB write); the events bracket the call alone
+        with ClockSampler(local) as clocks:
+            barrier(world)
+            torch.cuda.synchronize()
+            for i in range(Ks):
+                flush.fill_(i & 0xFF)
+                L.csa2_set_profile_events(4, ctypes.c_void_p(ev[i][0].cuda_event),
+                                          ctypes.c_void_p(ev[i][1].cuda_event))
+                call()
+                L.csa2_set_profile_events(4, None, None)
+            torch.cuda.synchronize()
+            barrier(world)
+        if int(err.item()):
+            raise RuntimeError(f"device error flags {int(err.item()):#x} during the benchmark")
+        call_ms = max_over_ranks(world, statistics.mean(a.elapsed_time(b) for a, b in ev), dev)
+        per_seq = K * 288 + W * 516
+        byts = B * per_seq
+        gbs = world * byts / (call_ms / 1e3) / 1e9
+        peak, peak_kind = measured_peak()
+        e2e = None
+        if not args.no_e2e:
+            q_h, idx_h = q.cpu().pin_memory(), idx.cpu().pin_memory()
+            out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+            lse_h = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+            ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(Ks)]
+            torch.cuda.synchronize()
+            for i in range(Ks):
+                flush.fill_(i & 0xFF)
+                ee[i][0].record(stream)
+                q.copy_(q_h, non_blocking=True)
+                idx.copy_(idx_h, non_blocking=True)
+                call()
+                out_h.copy_(out, non_blocking=True)
+                lse_h.copy_(lse, non_blocking=True)
+                ee[i][1].record(stream)
+            torch.cuda.synchronize()
+            e_ms = max_over_ranks(world, statistics.mean(a.elapsed_time(b) for a, b in ee), dev)
+            e2e = {"value": round(world * byts / (e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+                   "h2d_bytes_per_step": q.numel() * 2 + idx.numel() * 4,
+                   "d2h_bytes_per_step": out.numel() * 4 + lse.numel() * 4,
+                   "ms_per_step": round(e_ms, 5)}
+        cpu = None
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            cpu = sweep_cpu_baseline(wl, q, idx, dev)
+        line = {
+            "metric": SWEEP_METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": Ks, "warmup": Wu, "ms_per_step": round(call_ms, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp16-in fp32-acc (mxfp4 + fp8 cache)",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "B_per_gpu": B, "N": N, "K": K, "W": W,
+                       "indices": "512 uniform without replacement per sequence",
+                       "l2": "flushed before every call (256 MB write outside the events)",
+                       "parallelism": f"dp{world} (independent sequences)"},
+            "calls_per_s": round(world * 1e3 / call_ms, 1),
+            "roofline": {"kernel": "attend_kernel + attend_merge_kernel (one csa2_attend call)",
+                         "bound": "hbm", "achieved": round(byts / (call_ms / 1e3) / 1e9, 1),
+                         "peak": peak, "unit": "GB/s",
+                         "frac": round(byts / (call_ms / 1e3) / 1e9 / peak, 4),
+                         "peak_kind": peak_kind, "algorithmic_bytes_per_launch": byts,
+                         "algorithmic_bytes_per_sequence": per_seq,
+                         "launch_ms": round(call_ms, 5),
+                         "traffic": (lambda c: None if c is None else int(round(c["dram_bytes_per_sequence"] * B)))(
+                             captured_traffic("attend_reuse_traffic.json")),
+                         "timing": "CUDA events around every call, after an L2 flush"},
+            "gpu_launches": per_call_launches * Ks,
+            "clocks": clocks.summary(),
+        }
+        if e2e is not None:
+            line["e2e"] = e2e
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        del cache, ws
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
+    if args.steps is None and args.impl == "ours":
+        args.steps = 1000
     world, rank, local = dist_setup()
     try:
         if args.ced and args.impl == "ours":
@@ -1198,6 +1601,10 @@ def main():
             run_replay(args, world, rank, local)
         elif args.queries and args.impl == "ours":
             run_queries(args, world, rank, local)
+        elif args.append and args.impl == "ours":
+            run_append(args, world, rank, local)
+        elif args.sweep and args.impl == "ours":
+            run_sweep(args, world, rank, local)
         elif args.impl == "reference":
             run_reference(args, world, rank, local)
         else:

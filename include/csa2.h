@@ -235,7 +235,8 @@ CSA2_API int csa2_index_reindex(const void *iq, const float *w, const void *ik_c
  * CSA2_NOALLOC_REINDEX_MAX_SLOTS 8-byte slots (2 MiB) inside the library's device image, held by
  * every GPU that loads the library until the process exits; B * L above that limit returns
  * CSA2_ERR_UNSUPPORTED. The first call on a device looks up the array's device address for that
- * device (make that first call before any stream capture). All calls on a device share the
+ * device (make that first call before any stream capture); a call after the device's context was
+ * re-created (cudaDeviceReset) looks it up again. All calls on a device share the
  * array: calls whose kernels overlap on the GPU race and must be serialised by the caller. The
  * array needs no clearing: each call writes every slot it reads. It allocates nothing.
  */

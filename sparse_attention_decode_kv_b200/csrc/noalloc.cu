@@ -25,23 +25,53 @@ namespace {
 static __device__ __align__(256) uint64_t g_reindex_scratch[CSA2_NOALLOC_REINDEX_MAX_SLOTS];
 
 std::mutex g_scratch_mu;
-std::vector<void*> g_scratch_ptr;  // device address of g_reindex_scratch, per device
+// Device address of g_reindex_scratch, per device, with the context it was looked up in. A
+// device's primary context can be torn down and created again (cudaDeviceReset), which loads the
+// module afresh; the address is then looked up again.
+struct ScratchAddr {
+  void* ctx = nullptr;
+  void* ptr = nullptr;
+};
+std::vector<ScratchAddr> g_scratch;
 
-// The array's name is a host-side stand-in in host code; its device address is looked up once
-// per device, with that device current.
+// cuCtxGetCurrent from the driver, looked up once through the runtime (null if unavailable, in
+// which case the address is looked up on every call).
+using CtxGetCurrentFn = int (*)(void**);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(p);
+    return static_cast<CtxGetCurrentFn>(nullptr);
+  }();
+  return fn;
+}
+
+// The array's name is a host-side stand-in in host code; its device address is looked up at
+// set-up, once per device (and again if that device's context was re-created), with that device
+// current.
 cudaError_t scratch_for_current_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  // before the runtime has made a context current the answer is null, and the address is looked
+  // up (which makes it current) without being remembered
+  void* ctx = nullptr;
+  const CtxGetCurrentFn get = ctx_get_current();
+  const bool know_ctx = get != nullptr && get(&ctx) == 0 && ctx != nullptr;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (dev >= static_cast<int>(g_scratch_ptr.size())) g_scratch_ptr.resize(dev + 1, nullptr);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (dev >= static_cast<int>(g_scratch.size())) g_scratch.resize(dev + 1);
+  ScratchAddr& a = g_scratch[dev];
+  if (!know_ctx || a.ptr == nullptr || a.ctx != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_reindex_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
+    a.ptr = p;
+    a.ctx = know_ctx ? ctx : nullptr;
   }
-  *out = g_scratch_ptr[dev];
+  *out = a.ptr;
   return cudaSuccess;
 }
 

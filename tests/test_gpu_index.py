@@ -132,6 +132,34 @@ def test_full_index_candidates_beyond_shared_memory(gpu):
     assert list(pool[0]) == list(range(8 * P))
 
 
+@pytest.mark.parametrize("K,P,kind", [(4096, 2048, "gauss"), (512, 4096, "cluster"),
+                                      (4096, 4096, "ties"), (3000, 2100, "gauss")])
+def test_full_index_wide_selection(gpu, K, P, kind):
+    """max(K, P) above 2,048: the position Top-K runs over more than 16,384 positions (up to the
+    32,768 of 4,096 blocks), beyond what the selection keeps in registers, so the scores of the
+    wide blocks' positions are staged in shared memory."""
+    B, n_cap = 2, 40960
+    iq, w, ik = make_case(B, n_cap, seed=K + 3 * P, kind=kind)
+    N = [40960, 37003]
+    topk, pool, scores, err = run_full(iq, w, ik, N, K, P, gpu)
+    assert err == 0
+    check_full(iq, w, ik, N, K, P, topk, pool, scores)
+
+
+def test_full_index_wide_selection_all_equal(gpu):
+    """Every score equal and max(K, P) = 4,096: all 32,768 positions of the wide blocks fall in
+    the threshold bin, more candidates than the compaction buffer holds, so the select runs over
+    the staged keys themselves. Ties go to the lowest positions and blocks."""
+    B, n_cap, K, P = 1, 40960, 4096, 4096
+    iq = torch.zeros(B, 4, 64, dtype=torch.bfloat16)
+    w = torch.ones(B, 4)
+    ik = torch.randn(B, n_cap, 64).to(torch.bfloat16)
+    topk, pool, scores, err = run_full(iq, w, ik, [n_cap], K, P, gpu)
+    assert err == 0
+    assert list(topk[0]) == list(range(K))
+    assert list(pool[0]) == list(range(8 * P))
+
+
 @pytest.mark.parametrize("K,P", [(512, 16), (100, 7)])
 def test_full_index_pool_smaller_than_topk(gpu, K, P):
     """P < K: the Top-K comes from the top-K blocks while the pool keeps only the top P."""

@@ -58,6 +58,28 @@ def test_noalloc_reindex_matches_workspace_reindex_twice_in_a_row(gpu):
         assert np.array_equal(out.cpu().numpy(), ref.cpu().numpy())
 
 
+@pytest.mark.parametrize("B,n_cap,P", [(16, 16384, 2048), (8, 32768, 4096)])
+def test_noalloc_reindex_fills_its_whole_array(gpu, B, n_cap, P):
+    """B * L exactly the array's size: the last slot is written and read. The second case has
+    pools of 32,768 slots, above what the selection keeps in registers, so it reads its keys back
+    from the array on every pass."""
+    dev = gpu
+    K = 512
+    assert B * 8 * P == MAX_SLOTS
+    case = _case(3 + B, B, n_cap, K, P, dev)
+    ref = _reference(*case, K, dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    outs = []
+    for _ in range(2):
+        out = torch.full((B, K), -7, dtype=torch.int32, device=dev)
+        csa2.index_reindex_noalloc(*case, K, out, err)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    for out in outs:
+        assert np.array_equal(out.cpu().numpy(), ref.cpu().numpy())
+
+
 def test_noalloc_reindex_rejects_more_slots_than_its_array(gpu):
     dev = gpu
     B, L, K = 17, 16384, 64  # 278,528 slots > 262,144
