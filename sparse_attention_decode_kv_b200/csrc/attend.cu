@@ -609,7 +609,9 @@ __global__ void __launch_bounds__(128)
 
 int attend_split_count(int B, int K, int W) {
   const int tiles = (K + kTile - 1) / kTile + (W + kTile - 1) / kTile;
-  int splits = (kTargetCtas + B - 1) / B;
+  // at most one wave of two CTAs per SM: from 148 queries up every CTA takes whole queries and
+  // no partial outputs are written or merged
+  int splits = kTargetCtas / B;
   if (splits > tiles) splits = tiles;
   if (splits > kMaxSplits) splits = kMaxSplits;
   if (splits < 1) splits = 1;

@@ -15,7 +15,7 @@ itself.
 Checks:
 - MXFP4 bytes of sampled appended rows: bit for bit.
 - Attention of sampled sequences: within the output tolerance, on each batch size's own launch
-  shape (split counts 10, 10, 5 and 2 with the merge).
+  shape (10, 10 and 4 splits with the merge, one CTA per sequence at 256).
 """
 import numpy as np
 import pytest
