@@ -18,15 +18,16 @@
 //   block_collect_kernel  finds the histogram bin holding the max(K, P)-th block and copies the
 //                       rank keys of all blocks in or above it, in block order, into one region
 //                       per 8192-block chunk.
-//   index_final_kernel  one CTA per sequence: the top max(K, P) blocks among the candidates
-//                       (held in registers; the scan's histogram fixes the top 12 key bits, the
-//                       radix select refines them), an order-preserving compaction (ascending
-//                       block ids, no sort), the pool (top P blocks), then the position Top-K
-//                       over the positions of those blocks, selected the same way from the
-//                       gathered scores and a histogram built while gathering them. Every Top-K
-//                       position lies in one of the top max(K, P) blocks: a block ranked above
-//                       the block of a selected position holds its own maximum, which outranks
-//                       that position, so fewer than K blocks outrank it.
+//   index_final_kernel  two CTAs per sequence, running at once. The first selects the top P
+//                       blocks among the candidates (held in registers; the scan's histogram
+//                       fixes the top 12 key bits, the radix select refines them), compacts
+//                       them in order (ascending block ids, no sort) and writes the pool. The
+//                       second selects the top K blocks the same way, then the position Top-K
+//                       over their positions, from the gathered scores and a histogram built
+//                       while gathering them. Every Top-K position lies in one of the top K
+//                       blocks: a block ranked above the block of a selected position holds its
+//                       own maximum, which outranks that position, so fewer than K blocks
+//                       outrank it.
 // Every mbarrier wait is bounded; a timeout flags CSA2_DEVERR_TIMEOUT and the CTA drains its own
 // bulk copies before exiting.
 #include <mutex>
@@ -363,7 +364,9 @@ __global__ void __launch_bounds__(kFinalThreads)
   FinalSmem& sm = *reinterpret_cast<FinalSmem*>(smem_raw);
   pdl_wait();
   pdl_launch_dependents();
-  const int b = blockIdx.x, tid = threadIdx.x;
+  // role 0: the pool (top P blocks); role 1: the position Top-K, which needs nothing from role 0
+  // (both take their blocks from the candidates, which hold the top max(K, P) blocks)
+  const int b = blockIdx.x, role = blockIdx.y, tid = threadIdx.x;
   const int nb = max(0, min(__ldg(N + b), n_cap));
   const int nbl = (nb + S - 1) / S;
   const int kw = min(max(K, P), nbl);  // blocks that hold every Top-K position and the pool
@@ -374,12 +377,15 @@ __global__ void __launch_bounds__(kFinalThreads)
   int32_t* pool_out = pool + static_cast<int64_t>(b) * P * S;
   int32_t* topk_out = topk + static_cast<int64_t>(b) * K;
   if (kw == 0) {
-    for (int i = tid; i < P * S; i += kFinalThreads) pool_out[i] = -1;
-    for (int i = tid; i < K; i += kFinalThreads) topk_out[i] = -1;
+    if (role == 0)
+      for (int i = tid; i < P * S; i += kFinalThreads) pool_out[i] = -1;
+    else
+      for (int i = tid; i < K; i += kFinalThreads) topk_out[i] = -1;
     return;
   }
 
-  // ---- block candidates in block order
+  // ---- block candidates (every block whose maximum is in or above the bin of the kw-th one), in
+  // block order
   const uint32_t* cnts = ccnt + static_cast<int64_t>(b) * nchunks;
   const uint64_t* cbase = cand + static_cast<int64_t>(b) * nchunks * kCollectChunk;
   // prefix over chunk counts (thread c owns chunks 4c..4c+3)
@@ -414,174 +420,170 @@ __global__ void __launch_bounds__(kFinalThreads)
     return __ldg(cbase + static_cast<int64_t>(lo) * kCollectChunk + (i - sm.v.chunk_pre[lo]));
   };
 
-  // ---- top kw blocks, ascending
-  if (C <= kRegKeys * kFinalThreads) {
-    // Candidate 1024 j + t in thread t's key j. The scan's histogram of every block maximum
-    // fixes the top 12 bits of the kw-th key (the candidates are all blocks at or above that
-    // bin); the radix select goes on over the candidates in that bin.
-    for (int i = tid; i < kDigitBins; i += kFinalThreads) sm.u.r.fresh[i] = 0u;
-    uint64_t key[kRegKeys];
+  // ---- the top kx blocks among the candidates, ascending, into sm.wide / sm.wide_key
+  auto select_blocks = [&](int kx) {
+    if (C <= kRegKeys * kFinalThreads) {
+      // Candidate 1024 j + t in thread t's key j. The scan's histogram of every block maximum
+      // fixes the top 12 bits of the kx-th key (the candidates are all blocks at or above the
+      // bin of the kw-th one, kx <= kw); the radix select goes on over the candidates in that bin.
+      for (int i = tid; i < kDigitBins; i += kFinalThreads) sm.u.r.fresh[i] = 0u;
+      uint64_t key[kRegKeys];
 #pragma unroll
-    for (int j = 0; j < kRegKeys; ++j) {
-      const int i = j * kFinalThreads + tid;
-      key[j] = i < C ? cand_at(i) : 0ull;
+      for (int j = 0; j < kRegKeys; ++j) {
+        const int i = j * kFinalThreads + tid;
+        key[j] = i < C ? cand_at(i) : 0ull;
+      }
+      radix_state_from_top12(hist_g + static_cast<int64_t>(b) * kHistBins,
+                             static_cast<uint32_t>(kx), sm.sc);
+      block_radix_refine_visit(
+          [&](auto f) {
+#pragma unroll
+            for (int j = 0; j < kRegKeys; ++j) f(key[j]);
+          },
+          sm.u.r.fresh, sm.sc);
+      const RadixState st = sm.sc.st;
+      block_ordered_compact_regs16<false>(
+          [&](int j) { return key[j] != 0ull && radix_selected(key[j], st); },
+          [&](int j, uint32_t slot) {
+            if (slot < kMaxSel) {
+              sm.wide[slot] = static_cast<int32_t>(rank_key_index(key[j]));
+              sm.wide_key[slot] = key[j];
+            }
+          },
+          sm.u.r.wc);
+      __syncthreads();
+    } else {
+      block_radix_select(cand_at, C, static_cast<uint32_t>(kx), sm.sc);
+      const RadixState st = sm.sc.st;
+      block_ordered_compact(
+          C, [&](int i) { return radix_selected(cand_at(i), st); },
+          [&](int i, uint32_t slot) {
+            if (slot < kMaxSel) {
+              const uint64_t key = cand_at(i);
+              sm.wide[slot] = static_cast<int32_t>(rank_key_index(key));
+              sm.wide_key[slot] = key;
+            }
+          },
+          sm.sc.scan);
     }
-    radix_state_from_top12(hist_g + static_cast<int64_t>(b) * kHistBins, static_cast<uint32_t>(kw),
-                           sm.sc);
-    block_radix_refine_visit(
-        [&](auto f) {
-#pragma unroll
-          for (int j = 0; j < kRegKeys; ++j) f(key[j]);
-        },
-        sm.u.r.fresh, sm.sc);
-    const RadixState st = sm.sc.st;
-    block_ordered_compact_regs16<false>(
-        [&](int j) { return key[j] != 0ull && radix_selected(key[j], st); },
-        [&](int j, uint32_t slot) {
-          if (slot < kMaxSel) {
-            sm.wide[slot] = static_cast<int32_t>(rank_key_index(key[j]));
-            sm.wide_key[slot] = key[j];
-          }
-        },
-        sm.u.r.wc);
-    __syncthreads();
-  } else {
-    block_radix_select(cand_at, C, static_cast<uint32_t>(kw), sm.sc);
-    const RadixState st = sm.sc.st;
-    block_ordered_compact(
-        C, [&](int i) { return radix_selected(cand_at(i), st); },
-        [&](int i, uint32_t slot) {
-          if (slot < kMaxSel) {
-            const uint64_t key = cand_at(i);
-            sm.wide[slot] = static_cast<int32_t>(rank_key_index(key));
-            sm.wide_key[slot] = key;
-          }
-        },
-        sm.sc.scan);
-  }
-  // ---- the pool: the top kp blocks, i.e. the whole wide set unless P < K
-  const uint64_t* wk = sm.wide_key;
-  if (kp < kw) {
-    auto wide_key = [wk](int i) { return wk[i]; };
-    block_radix_select(wide_key, kw, static_cast<uint32_t>(kp), sm.sc);
-    const RadixState st = sm.sc.st;
-    const uint32_t n_pool = block_ordered_compact(
-        kw, [&](int i) { return radix_selected(wk[i], st); },
-        [&](int i, uint32_t slot) {
-          for (int r = 0; r < S; ++r) {
-            const int p = sm.wide[i] * S + r;
-            pool_out[slot * S + r] = p < nb ? p : -1;
-          }
-        },
-        sm.sc.scan);
-    for (int i = static_cast<int>(n_pool) * S + tid; i < P * S; i += kFinalThreads)
-      pool_out[i] = -1;
-  } else {
+  };
+
+  if (role == 0) {
+    // ---- the pool: the top kp blocks, ascending, expanded to their positions
+    select_blocks(kp);
     for (int i = tid; i < P * S; i += kFinalThreads) {
       const int j = i / S;
-      const int p = j < kw ? sm.wide[j] * S + (i % S) : nb;
+      const int p = j < kp ? sm.wide[j] * S + (i % S) : nb;
       pool_out[i] = p < nb ? p : -1;
     }
+    return;
   }
 
-  // ---- position Top-K over every position of the wide blocks (item i = position i % 8 of block
-  // wide[i / 8]: ascending positions). The score gather also histograms the top 12 bits of each
-  // rank key, which fixes those bits of the K-th key; the radix select continues from there.
-  const int L = kw * S;  // <= 32768
   const float* srow = scores + static_cast<int64_t>(b) * n_cap;
-  uint32_t n_sel;
-  if (L <= kRegKeys * kFinalThreads) {
-    // position item 1024 j + t in thread t's key j (0: past N or past the wide blocks)
-    for (int i = tid; i < kDigitBins; i += kFinalThreads) {
-      sm.sc.hist[i] = 0u;
-      sm.u.r.fresh[i] = 0u;
-    }
-    __syncthreads();
-    // all score loads first: the high word holds the raw score bits until they land, the low
-    // word the inverted position (never 0 for a real position)
-    uint32_t hi[kRegKeys], lo[kRegKeys];
-#pragma unroll
-    for (int j = 0; j < kRegKeys; ++j) {
-      const int i = j * kFinalThreads + tid;
-      const int p = i < L ? sm.wide[i / S] * S + (i % S) : nb;
-      lo[j] = p < nb ? ~static_cast<uint32_t>(p) : 0u;
-      hi[j] = p < nb ? __float_as_uint(__ldg(srow + p)) : 0u;
-    }
-    uint64_t key[kRegKeys];
-#pragma unroll
-    for (int j = 0; j < kRegKeys; ++j) {
-      key[j] = lo[j] != 0u ? rank_key(__uint_as_float(hi[j]), ~lo[j]) : 0ull;
-      if (key[j] != 0ull) atomicAdd(&sm.sc.hist[static_cast<uint32_t>(key[j] >> 52)], 1u);
-    }
-    __syncthreads();
-    radix_state_from_top12(sm.sc.hist, static_cast<uint32_t>(kk), sm.sc);
-    block_radix_refine_visit(
-        [&](auto f) {
-#pragma unroll
-          for (int j = 0; j < kRegKeys; ++j) f(key[j]);
-        },
-        sm.u.r.fresh, sm.sc);
-    const RadixState st = sm.sc.st;
-    n_sel = block_ordered_compact_regs16<false>(
-        [&](int j) { return key[j] != 0ull && radix_selected(key[j], st); },
-        [&](int j, uint32_t slot) {
-          if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(rank_key_index(key[j]));
-        },
-        sm.u.r.wc);
-  } else {
-    for (int i = tid; i < kDigitBins; i += kFinalThreads) sm.sc.hist[i] = 0u;
-    __syncthreads();
-    for (int base = 0; base < L; base += 8 * kFinalThreads) {
-      float vals[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = base + j * kFinalThreads + tid;
-        const int p = i < L ? sm.wide[i / S] * S + (i % S) : nb;
-        vals[j] = p < nb ? __ldg(srow + p) : 0.0f;
+  uint32_t n_sel = 0;
+  {
+    // ---- the position Top-K: the top kq blocks, then the Top-K over their positions. A block
+    // ranked above the block of a Top-K position holds its own maximum, which outranks that
+    // position, so fewer than K blocks outrank it: every Top-K position lies in the top K blocks.
+    const int kq = min(K, nbl);
+    select_blocks(kq);
+    // position Top-K over every position of those blocks (item i = position i % 8 of block
+    // wide[i / 8]: ascending positions). The score gather also histograms the top 12 bits of each
+    // rank key, which fixes those bits of the K-th key; the radix select continues from there.
+    const int L = kq * S;  // <= 32768
+    if (L <= kRegKeys * kFinalThreads) {
+      // position item 1024 j + t in thread t's key j (0: past N or past the wide blocks)
+      for (int i = tid; i < kDigitBins; i += kFinalThreads) {
+        sm.sc.hist[i] = 0u;
+        sm.u.r.fresh[i] = 0u;
       }
+      __syncthreads();
+      // all score loads first: the high word holds the raw score bits until they land, the low
+      // word the inverted position (never 0 for a real position)
+      uint32_t hi[kRegKeys], lo[kRegKeys];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = base + j * kFinalThreads + tid;
-        if (i < L) {
-          const int p = sm.wide[i / S] * S + (i % S);
-          const uint32_t key = p < nb ? float_key(vals[j]) : 0u;  // 0: below every real key
-          sm.u.skey[i] = key;
-          if (p < nb) atomicAdd(&sm.sc.hist[key >> kHistShift], 1u);
+      for (int j = 0; j < kRegKeys; ++j) {
+        const int i = j * kFinalThreads + tid;
+        const int p = i < L ? sm.wide[i / S] * S + (i % S) : nb;
+        lo[j] = p < nb ? ~static_cast<uint32_t>(p) : 0u;
+        hi[j] = p < nb ? __float_as_uint(__ldg(srow + p)) : 0u;
+      }
+      uint64_t key[kRegKeys];
+#pragma unroll
+      for (int j = 0; j < kRegKeys; ++j) {
+        key[j] = lo[j] != 0u ? rank_key(__uint_as_float(hi[j]), ~lo[j]) : 0ull;
+        if (key[j] != 0ull) atomicAdd(&sm.sc.hist[static_cast<uint32_t>(key[j] >> 52)], 1u);
+      }
+      __syncthreads();
+      radix_state_from_top12(sm.sc.hist, static_cast<uint32_t>(kk), sm.sc);
+      block_radix_refine_visit(
+          [&](auto f) {
+#pragma unroll
+            for (int j = 0; j < kRegKeys; ++j) f(key[j]);
+          },
+          sm.u.r.fresh, sm.sc);
+      const RadixState st = sm.sc.st;
+      n_sel = block_ordered_compact_regs16<false>(
+          [&](int j) { return key[j] != 0ull && radix_selected(key[j], st); },
+          [&](int j, uint32_t slot) {
+            if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(rank_key_index(key[j]));
+          },
+          sm.u.r.wc);
+    } else {
+      for (int i = tid; i < kDigitBins; i += kFinalThreads) sm.sc.hist[i] = 0u;
+      __syncthreads();
+      for (int base = 0; base < L; base += 8 * kFinalThreads) {
+        float vals[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = base + j * kFinalThreads + tid;
+          const int p = i < L ? sm.wide[i / S] * S + (i % S) : nb;
+          vals[j] = p < nb ? __ldg(srow + p) : 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = base + j * kFinalThreads + tid;
+          if (i < L) {
+            const int p = sm.wide[i / S] * S + (i % S);
+            const uint32_t key = p < nb ? float_key(vals[j]) : 0u;  // 0: below every real key
+            sm.u.skey[i] = key;
+            if (p < nb) atomicAdd(&sm.sc.hist[key >> kHistShift], 1u);
+          }
         }
       }
-    }
-    __syncthreads();
-    auto pos_of = [&](int i) { return static_cast<uint32_t>(sm.wide[i / S] * S + (i % S)); };
-    auto pos_key = [&](int i) -> uint64_t {
-      const uint32_t hk = sm.u.skey[i];
-      return hk == 0u ? 0ull : (static_cast<uint64_t>(hk) << 32) | static_cast<uint64_t>(~pos_of(i));
-    };
-    const int T0 = block_find_bin4096(sm.sc.hist, static_cast<uint32_t>(kk), sm.sc.part, sm.sc.ints);
-    // candidates in slot order into the (now free) wide_key array
-    uint64_t* cbuf = sm.wide_key;
-    const uint32_t n_cand = block_ordered_compact(
-        L, [&](int i) { const uint32_t k = sm.u.skey[i]; return k != 0u && static_cast<int>(k >> kHistShift) >= T0; },
-        [&](int i, uint32_t slot) { if (slot < kMaxSel) cbuf[slot] = pos_key(i); }, sm.sc.scan);
-    __syncthreads();
-    if (n_cand <= static_cast<uint32_t>(kMaxSel)) {
-      auto get = [cbuf](int i) { return cbuf[i]; };
-      block_radix_select(get, static_cast<int>(n_cand), static_cast<uint32_t>(kk), sm.sc);
-      const RadixState st = sm.sc.st;
-      n_sel = block_ordered_compact(
-          static_cast<int>(n_cand), [&](int i) { return radix_selected(cbuf[i], st); },
-          [&](int i, uint32_t slot) {
-            if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(rank_key_index(cbuf[i]));
-          },
-          sm.sc.scan);
-    } else {
-      block_radix_select(pos_key, L, static_cast<uint32_t>(kk), sm.sc);
-      const RadixState st = sm.sc.st;
-      n_sel = block_ordered_compact(
-          L, [&](int i) { const uint64_t k = pos_key(i); return k != 0ull && radix_selected(k, st); },
-          [&](int i, uint32_t slot) {
-            if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(pos_of(i));
-          },
-          sm.sc.scan);
+      __syncthreads();
+      auto pos_of = [&](int i) { return static_cast<uint32_t>(sm.wide[i / S] * S + (i % S)); };
+      auto pos_key = [&](int i) -> uint64_t {
+        const uint32_t hk = sm.u.skey[i];
+        return hk == 0u ? 0ull : (static_cast<uint64_t>(hk) << 32) | static_cast<uint64_t>(~pos_of(i));
+      };
+      const int T0 = block_find_bin4096(sm.sc.hist, static_cast<uint32_t>(kk), sm.sc.part, sm.sc.ints);
+      // candidates in slot order into the (now free) wide_key array
+      uint64_t* cbuf = sm.wide_key;
+      const uint32_t n_cand = block_ordered_compact(
+          L, [&](int i) { const uint32_t k = sm.u.skey[i]; return k != 0u && static_cast<int>(k >> kHistShift) >= T0; },
+          [&](int i, uint32_t slot) { if (slot < kMaxSel) cbuf[slot] = pos_key(i); }, sm.sc.scan);
+      __syncthreads();
+      if (n_cand <= static_cast<uint32_t>(kMaxSel)) {
+        auto get = [cbuf](int i) { return cbuf[i]; };
+        block_radix_select(get, static_cast<int>(n_cand), static_cast<uint32_t>(kk), sm.sc);
+        const RadixState st = sm.sc.st;
+        n_sel = block_ordered_compact(
+            static_cast<int>(n_cand), [&](int i) { return radix_selected(cbuf[i], st); },
+            [&](int i, uint32_t slot) {
+              if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(rank_key_index(cbuf[i]));
+            },
+            sm.sc.scan);
+      } else {
+        block_radix_select(pos_key, L, static_cast<uint32_t>(kk), sm.sc);
+        const RadixState st = sm.sc.st;
+        n_sel = block_ordered_compact(
+            L, [&](int i) { const uint64_t k = pos_key(i); return k != 0ull && radix_selected(k, st); },
+            [&](int i, uint32_t slot) {
+              if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(pos_of(i));
+            },
+            sm.sc.scan);
+      }
     }
   }
   for (int i = static_cast<int>(n_sel) + tid; i < K; i += kFinalThreads) topk_out[i] = -1;
@@ -890,7 +892,7 @@ cudaError_t launch_index_full(const void* iq, const float* w, const void* ik_cac
                  static_cast<const uint32_t*>(hist), ccnt, cand);
   count_launches(1);
   if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
-  e = launch_pdl(index_final_kernel, dim3(B), dim3(kFinalThreads), sizeof(FinalSmem), s,
+  e = launch_pdl(index_final_kernel, dim3(B, 2), dim3(kFinalThreads), sizeof(FinalSmem), s,
                  static_cast<const float*>(scores), N, n_cap, K, P,
                  static_cast<const uint32_t*>(hist), static_cast<const uint32_t*>(ccnt),
                  static_cast<const uint64_t*>(cand), topk, pool);
