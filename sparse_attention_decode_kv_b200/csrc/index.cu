@@ -31,6 +31,7 @@
 // Every mbarrier wait is bounded; a timeout flags CSA2_DEVERR_TIMEOUT and the CTA drains its own
 // bulk copies before exiting.
 #include <mutex>
+#include <type_traits>
 #include <vector>
 
 #include "common.cuh"
@@ -420,38 +421,45 @@ __global__ void __launch_bounds__(kFinalThreads)
     return __ldg(cbase + static_cast<int64_t>(lo) * kCollectChunk + (i - sm.v.chunk_pre[lo]));
   };
 
-  // ---- the top kx blocks among the candidates, ascending, into sm.wide / sm.wide_key
+  // ---- the top kx blocks among the candidates, ascending, into sm.wide / sm.wide_key.
+  // Candidate 1024 j + t in thread t's key j (NK keys per thread: 4 when they fit, else 16). The
+  // scan's histogram of every block maximum fixes the top 12 bits of the kx-th key (the
+  // candidates are all blocks at or above the bin of the kw-th one, kx <= kw); the radix select
+  // goes on over the candidates in that bin.
+  auto select_blocks_regs = [&](auto nk, int kx) {
+    constexpr int NK = decltype(nk)::value;
+    for (int i = tid; i < kDigitBins; i += kFinalThreads) sm.u.r.fresh[i] = 0u;
+    uint64_t key[NK];
+#pragma unroll
+    for (int j = 0; j < NK; ++j) {
+      const int i = j * kFinalThreads + tid;
+      key[j] = i < C ? cand_at(i) : 0ull;
+    }
+    radix_state_from_top12(hist_g + static_cast<int64_t>(b) * kHistBins, static_cast<uint32_t>(kx),
+                           sm.sc);
+    block_radix_refine_visit(
+        [&](auto f) {
+#pragma unroll
+          for (int j = 0; j < NK; ++j) f(key[j]);
+        },
+        sm.u.r.fresh, sm.sc);
+    const RadixState st = sm.sc.st;
+    block_ordered_compact_regs<NK, false>(
+        [&](int j) { return key[j] != 0ull && radix_selected(key[j], st); },
+        [&](int j, uint32_t slot) {
+          if (slot < kMaxSel) {
+            sm.wide[slot] = static_cast<int32_t>(rank_key_index(key[j]));
+            sm.wide_key[slot] = key[j];
+          }
+        },
+        sm.u.r.wc);
+    __syncthreads();
+  };
   auto select_blocks = [&](int kx) {
-    if (C <= kRegKeys * kFinalThreads) {
-      // Candidate 1024 j + t in thread t's key j. The scan's histogram of every block maximum
-      // fixes the top 12 bits of the kx-th key (the candidates are all blocks at or above the
-      // bin of the kw-th one, kx <= kw); the radix select goes on over the candidates in that bin.
-      for (int i = tid; i < kDigitBins; i += kFinalThreads) sm.u.r.fresh[i] = 0u;
-      uint64_t key[kRegKeys];
-#pragma unroll
-      for (int j = 0; j < kRegKeys; ++j) {
-        const int i = j * kFinalThreads + tid;
-        key[j] = i < C ? cand_at(i) : 0ull;
-      }
-      radix_state_from_top12(hist_g + static_cast<int64_t>(b) * kHistBins,
-                             static_cast<uint32_t>(kx), sm.sc);
-      block_radix_refine_visit(
-          [&](auto f) {
-#pragma unroll
-            for (int j = 0; j < kRegKeys; ++j) f(key[j]);
-          },
-          sm.u.r.fresh, sm.sc);
-      const RadixState st = sm.sc.st;
-      block_ordered_compact_regs16<false>(
-          [&](int j) { return key[j] != 0ull && radix_selected(key[j], st); },
-          [&](int j, uint32_t slot) {
-            if (slot < kMaxSel) {
-              sm.wide[slot] = static_cast<int32_t>(rank_key_index(key[j]));
-              sm.wide_key[slot] = key[j];
-            }
-          },
-          sm.u.r.wc);
-      __syncthreads();
+    if (C <= 4 * kFinalThreads) {
+      select_blocks_regs(std::integral_constant<int, 4>{}, kx);
+    } else if (C <= kRegKeys * kFinalThreads) {
+      select_blocks_regs(std::integral_constant<int, kRegKeys>{}, kx);
     } else {
       block_radix_select(cand_at, C, static_cast<uint32_t>(kx), sm.sc);
       const RadixState st = sm.sc.st;
@@ -491,8 +499,10 @@ __global__ void __launch_bounds__(kFinalThreads)
     // wide[i / 8]: ascending positions). The score gather also histograms the top 12 bits of each
     // rank key, which fixes those bits of the K-th key; the radix select continues from there.
     const int L = kq * S;  // <= 32768
-    if (L <= kRegKeys * kFinalThreads) {
-      // position item 1024 j + t in thread t's key j (0: past N or past the wide blocks)
+    // position item 1024 j + t in thread t's key j (NK keys per thread: 4 when they fit, else
+    // 16; key 0: past N or past the blocks)
+    auto positions_regs = [&](auto nk) -> uint32_t {
+      constexpr int NK = decltype(nk)::value;
       for (int i = tid; i < kDigitBins; i += kFinalThreads) {
         sm.sc.hist[i] = 0u;
         sm.u.r.fresh[i] = 0u;
@@ -500,17 +510,17 @@ __global__ void __launch_bounds__(kFinalThreads)
       __syncthreads();
       // all score loads first: the high word holds the raw score bits until they land, the low
       // word the inverted position (never 0 for a real position)
-      uint32_t hi[kRegKeys], lo[kRegKeys];
+      uint32_t hi[NK], lo[NK];
 #pragma unroll
-      for (int j = 0; j < kRegKeys; ++j) {
+      for (int j = 0; j < NK; ++j) {
         const int i = j * kFinalThreads + tid;
         const int p = i < L ? sm.wide[i / S] * S + (i % S) : nb;
         lo[j] = p < nb ? ~static_cast<uint32_t>(p) : 0u;
         hi[j] = p < nb ? __float_as_uint(__ldg(srow + p)) : 0u;
       }
-      uint64_t key[kRegKeys];
+      uint64_t key[NK];
 #pragma unroll
-      for (int j = 0; j < kRegKeys; ++j) {
+      for (int j = 0; j < NK; ++j) {
         key[j] = lo[j] != 0u ? rank_key(__uint_as_float(hi[j]), ~lo[j]) : 0ull;
         if (key[j] != 0ull) atomicAdd(&sm.sc.hist[static_cast<uint32_t>(key[j] >> 52)], 1u);
       }
@@ -519,16 +529,21 @@ __global__ void __launch_bounds__(kFinalThreads)
       block_radix_refine_visit(
           [&](auto f) {
 #pragma unroll
-            for (int j = 0; j < kRegKeys; ++j) f(key[j]);
+            for (int j = 0; j < NK; ++j) f(key[j]);
           },
           sm.u.r.fresh, sm.sc);
       const RadixState st = sm.sc.st;
-      n_sel = block_ordered_compact_regs16<false>(
+      return block_ordered_compact_regs<NK, false>(
           [&](int j) { return key[j] != 0ull && radix_selected(key[j], st); },
           [&](int j, uint32_t slot) {
             if (slot < static_cast<uint32_t>(K)) topk_out[slot] = static_cast<int32_t>(rank_key_index(key[j]));
           },
           sm.u.r.wc);
+    };
+    if (L <= 4 * kFinalThreads) {
+      n_sel = positions_regs(std::integral_constant<int, 4>{});
+    } else if (L <= kRegKeys * kFinalThreads) {
+      n_sel = positions_regs(std::integral_constant<int, kRegKeys>{});
     } else {
       for (int i = tid; i < kDigitBins; i += kFinalThreads) sm.sc.hist[i] = 0u;
       __syncthreads();

@@ -316,32 +316,34 @@ __device__ uint32_t block_ordered_compact(int n, const Pred& pred, const Emit& e
 }
 
 // Order-preserving compaction over items held in registers by a CTA of 1,024 threads: thread t
-// holds item 1024 j + t in its slot j (j < 16). emit(j, slot) runs for each item with sel(j),
-// slot counting the selected items in item order. The (slot, warp) counts are published in item
-// order and every warp takes its offsets from them after one barrier. wc: 544 shared words (512
-// counts, one pad word after every 16 so that a lane's 16 reads hit distinct banks). Returns the
-// count; the caller synchronises before emitted data is read by other threads or wc is reused.
-// kKeepMasks: keep the 16 ballot masks in registers across the barrier, or form them again after
-// it (for callers short of registers).
-template <bool kKeepMasks, class Sel, class Emit>
-__device__ uint32_t block_ordered_compact_regs16(const Sel& sel, const Emit& emit, uint32_t* wc) {
+// holds item 1024 j + t in its slot j (j < NK, NK = 4 or 16). emit(j, slot) runs for each item
+// with sel(j), slot counting the selected items in item order. The (slot, warp) counts are
+// published in item order and every warp takes its offsets from them after one barrier. wc: 544
+// shared words (32 NK counts, one pad word after every 16 so that a lane's reads hit distinct
+// banks). Returns the count; the caller synchronises before emitted data is read by other
+// threads or wc is reused. kKeepMasks: keep the NK ballot masks in registers across the barrier,
+// or form them again after it (for callers short of registers).
+template <int NK, bool kKeepMasks, class Sel, class Emit>
+__device__ uint32_t block_ordered_compact_regs(const Sel& sel, const Emit& emit, uint32_t* wc) {
+  static_assert(NK == 4 || NK == 16, "4 or 16 items per thread");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t mk[16];
+  uint32_t mk[NK];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
+  for (int j = 0; j < NK; ++j) {
     const uint32_t m = __ballot_sync(0xFFFFFFFFu, sel(j));
     if (kKeepMasks) mk[j] = m;
     const int e = 32 * j + warp;  // item order of (slot j, warp)
     if (lane == 0) wc[e + (e >> 4)] = static_cast<uint32_t>(__popc(m));
   }
   __syncthreads();
-  // lane l holds entries 16 l .. 16 l + 15; this warp's entries sit at offset warp & 15 of lanes
-  // 2 j + (warp >> 4)
+  // lane l holds entries NK l .. NK l + NK - 1; this warp's entries sit at offset warp % NK of
+  // lanes (32 / NK) j + warp / NK
   uint32_t lsum = 0, lpre = 0;
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const uint32_t cq = wc[17 * lane + q];
-    lpre += q < (warp & 15) ? cq : 0u;
+  for (int q = 0; q < NK; ++q) {
+    const int e = NK * lane + q;
+    const uint32_t cq = wc[e + (e >> 4)];
+    lpre += q < (warp % NK) ? cq : 0u;
     lsum += cq;
   }
   uint32_t incl = lsum;
@@ -354,12 +356,17 @@ __device__ uint32_t block_ordered_compact_regs16(const Sel& sel, const Emit& emi
   const uint32_t mine = incl - lsum + lpre;
   const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const uint32_t base = __shfl_sync(0xFFFFFFFFu, mine, 2 * j + (warp >> 4));
+  for (int j = 0; j < NK; ++j) {
+    const uint32_t base = __shfl_sync(0xFFFFFFFFu, mine, (32 / NK) * j + warp / NK);
     const uint32_t m = kKeepMasks ? mk[j] : __ballot_sync(0xFFFFFFFFu, sel(j));
     if ((m >> lane) & 1u) emit(j, base + static_cast<uint32_t>(__popc(m & lt)));
   }
   return total;
+}
+
+template <bool kKeepMasks, class Sel, class Emit>
+__device__ uint32_t block_ordered_compact_regs16(const Sel& sel, const Emit& emit, uint32_t* wc) {
+  return block_ordered_compact_regs<16, kKeepMasks>(sel, emit, wc);
 }
 
 // Ascending bitonic sort of a[0..n2) in shared memory, n2 a power of two (whole CTA).
