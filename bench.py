@@ -91,6 +91,8 @@ def parse():
                     help="measure Reuse-mode attention at the sweep's batch sizes (one line each)")
     ap.add_argument("--sweep-batches", default="1,8,64,256",
                     help="batch sizes of --sweep (default 1,8,64,256)")
+    ap.add_argument("--sweep-n", type=int, default=131072,
+                    help="cached entries per sequence for --sweep (default 131,072)")
     ap.add_argument("--breakdown", action="store_true",
                     help="also time each library call of the step (eager, synchronised)")
     return ap.parse_args()
@@ -1259,7 +1261,7 @@ def run_replay(args, world, rank, local):
 APPEND_METRIC = ("MXFP4 quantize-append GB/s (bf16 rows read + E2M1 codes and E4M3 scales written), "
                  "1,048,576 entries, 1 B200")
 SWEEP_METRIC = ("Reuse-mode sparse attention GB/s (gathered MXFP4 entries + FP8 SWA rows), "
-                "N=131,072, 1 B200")
+                "N={N:,}, 1 B200")
 L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
 
 
@@ -1484,8 +1486,9 @@ def run_sweep(args, world, rank, local):
     batches = [int(v) for v in args.sweep_batches.split(",")]
     for B in batches:
         base = next((w for w in workloads.REUSE_SWEEP if w.B == B), None)
-        if base is None:
-            base = workloads.ReuseAttendWorkload(f"reuse-attend-B{B}-N131072", B=B)
+        if base is None or args.sweep_n != base.N:
+            base = workloads.ReuseAttendWorkload(f"reuse-attend-B{B}-N{args.sweep_n}", B=B,
+                                                 N=args.sweep_n)
         wl = dataclasses.replace(base, seed=base.seed + 1000 * rank)
         N, K, W = wl.N, wl.K, wl.W
         cache = csa2.Cache(B, N, W, device=dev)
@@ -1563,7 +1566,7 @@ def run_sweep(args, world, rank, local):
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             cpu = sweep_cpu_baseline(wl, q, idx, dev)
         line = {
-            "metric": SWEEP_METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world,
+            "metric": SWEEP_METRIC.format(N=N), "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world,
             "steps": Ks, "warmup": Wu, "ms_per_step": round(call_ms, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "fp16-in fp32-acc (mxfp4 + fp8 cache)",
             "data": "synthetic",
