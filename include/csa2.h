@@ -252,11 +252,13 @@ CSA2_API int csa2_index_reindex_noalloc(const void *iq, const float *w, const vo
  * FP8 SWA KV. `mode` records which kind of layer produced idx; it does not change the result
  * (attend(REUSE, idx) == attend(FULL, idx) bit for bit). A Reuse layer's indices, and the cache
  * rows they name, were produced by an earlier layer, so with CSA2_MODE_REUSE the kernel starts
- * gathering them before it waits for the preceding kernel on the stream. The caller guarantees
- * that the immediately preceding call of this library on the stream writes neither idx nor the
- * codes and scales of the entries idx names. In a decode step that call is the previous layer's
- * csa2_attend, which writes only out, lse and its workspace. Use CSA2_MODE_FULL or
- * CSA2_MODE_REINDEX right after the call that produced idx or appended the entries.
+ * gathering them before it waits for the preceding kernel on the stream. It does so only when
+ * the library's previous call on the same stream was csa2_attend or csa2_attend_queries (which
+ * write only out, lse and their workspace), as in a decode step's run of Reuse layers; after any
+ * other call of the library on the stream (an append, an index call, a CED projection, a cache
+ * restore or a replay, which may write idx or the rows) it waits first. The library sees only
+ * its own calls: the caller guarantees that no other code on the stream writes idx or the
+ * entries' codes and scales between that attention and this one.
  *   q         bf16 [B, 16, 512]; every |q| must be below 65504 (fp16 range).
  *   codes/scales as written by csa2_append_quant; N int32 [B] (device).
  *   idx       int32 [B, K]: entry positions, -1 = none; duplicates count as separate entries.

@@ -4,6 +4,7 @@
 // call returns a status without launching anything (and works on a machine without a GPU).
 #include <atomic>
 #include <mutex>
+#include <unordered_map>
 #include <vector>
 
 #include "common.cuh"
@@ -37,6 +38,20 @@ TensorMapEncodeFn tensor_map_encoder() {
       fn = reinterpret_cast<TensorMapEncodeFn>(p);
   });
   return fn;
+}
+
+static std::mutex g_last_mu;
+static std::unordered_map<const void*, bool> g_last_attend;
+
+void note_call(cudaStream_t s, bool is_attend) {
+  std::lock_guard<std::mutex> lock(g_last_mu);
+  g_last_attend[static_cast<const void*>(s)] = is_attend;
+}
+
+bool last_call_was_attend(cudaStream_t s) {
+  std::lock_guard<std::mutex> lock(g_last_mu);
+  const auto it = g_last_attend.find(static_cast<const void*>(s));
+  return it != g_last_attend.end() && it->second;
 }
 
 int device_sm_count() {
@@ -148,9 +163,11 @@ int csa2_append_quant(const void* x, const void* ik, int B, int n, const int32_t
   if (!ring && W != 0) return CSA2_ERR_INVALID;
   if (dev_err != nullptr && (reinterpret_cast<uintptr_t>(dev_err) & 3u)) return CSA2_ERR_INVALID;
   if (n == 0) return CSA2_OK;
-  return cuda_status(csa2::launch_append(x, ik, B, n, pos, n_cap, codes, scales, ik_cache, swa,
+  const cudaError_t launch_err = csa2::launch_append(x, ik, B, n, pos, n_cap, codes, scales, ik_cache, swa,
                                          swa_scale, W, dev_err,
-                                         reinterpret_cast<cudaStream_t>(stream)));
+                                         reinterpret_cast<cudaStream_t>(stream));
+  csa2::note_call(reinterpret_cast<cudaStream_t>(stream), false);
+  return cuda_status(launch_err);
 }
 
 int csa2_ced_project_quant(const void* h, const void* w, int B, int n, int d, const int32_t* pos,
@@ -165,8 +182,10 @@ int csa2_ced_project_quant(const void* h, const void* w, int B, int n, int d, co
     return CSA2_ERR_INVALID;
   if (dev_err != nullptr && (reinterpret_cast<uintptr_t>(dev_err) & 3u)) return CSA2_ERR_INVALID;
   if (n == 0) return CSA2_OK;
-  return cuda_status(csa2::launch_ced_quant(h, w, B, n, d, pos, n_cap, codes, scales, dev_err,
-                                            reinterpret_cast<cudaStream_t>(stream)));
+  const cudaError_t launch_err = csa2::launch_ced_quant(h, w, B, n, d, pos, n_cap, codes, scales, dev_err,
+                                            reinterpret_cast<cudaStream_t>(stream));
+  csa2::note_call(reinterpret_cast<cudaStream_t>(stream), false);
+  return cuda_status(launch_err);
 }
 
 size_t csa2_index_full_workspace_bytes(int B, int n_cap, int K, int P) {
@@ -185,8 +204,10 @@ int csa2_index_full(const void* iq, const float* w, const void* ik_cache, const 
     return CSA2_ERR_INVALID;
   if (dev_err != nullptr && (reinterpret_cast<uintptr_t>(dev_err) & 3u)) return CSA2_ERR_INVALID;
   if (ws_bytes < csa2::index_full_workspace_bytes(B, n_cap, K, P)) return CSA2_ERR_WORKSPACE;
-  return cuda_status(csa2::launch_index_full(iq, w, ik_cache, N, B, n_cap, K, P, topk, pool, ws,
-                                             dev_err, reinterpret_cast<cudaStream_t>(stream)));
+  const cudaError_t launch_err = csa2::launch_index_full(iq, w, ik_cache, N, B, n_cap, K, P, topk, pool, ws,
+                                             dev_err, reinterpret_cast<cudaStream_t>(stream));
+  csa2::note_call(reinterpret_cast<cudaStream_t>(stream), false);
+  return cuda_status(launch_err);
 }
 
 size_t csa2_index_reindex_workspace_bytes(int B, int L, int K) {
@@ -205,9 +226,11 @@ int csa2_index_reindex(const void* iq, const float* w, const void* ik_cache, con
     return CSA2_ERR_INVALID;
   if (dev_err != nullptr && (reinterpret_cast<uintptr_t>(dev_err) & 3u)) return CSA2_ERR_INVALID;
   if (ws_bytes < csa2::index_reindex_workspace_bytes(B, L, K)) return CSA2_ERR_WORKSPACE;
-  return cuda_status(csa2::launch_index_reindex(iq, w, ik_cache, N, B, n_cap, pool, L, K, topk,
+  const cudaError_t launch_err = csa2::launch_index_reindex(iq, w, ik_cache, N, B, n_cap, pool, L, K, topk,
                                                 ws, dev_err,
-                                                reinterpret_cast<cudaStream_t>(stream)));
+                                                reinterpret_cast<cudaStream_t>(stream));
+  csa2::note_call(reinterpret_cast<cudaStream_t>(stream), false);
+  return cuda_status(launch_err);
 }
 
 size_t csa2_attend_workspace_bytes(int B, int K, int W) {
@@ -233,11 +256,15 @@ int csa2_attend(int mode, const void* q, float softmax_scale, const uint8_t* cod
   if (dev_err != nullptr && (reinterpret_cast<uintptr_t>(dev_err) & 3u)) return CSA2_ERR_INVALID;
   const size_t need = csa2::attend_workspace_bytes(B, K, W);
   if (need > 0 && (ws == nullptr || !aligned16(ws) || ws_bytes < need)) return CSA2_ERR_WORKSPACE;
-  return cuda_status(csa2::launch_attend(q, softmax_scale, codes, scales, n_cap, N, idx, K,
+  const cudaError_t launch_err = csa2::launch_attend(q, softmax_scale, codes, scales, n_cap, N, idx, K,
                                          W > 0 ? swa : nullptr, W > 0 ? swa_scale : nullptr,
                                          W > 0 ? swa_len : nullptr, W, nullptr, nullptr, W, B, B,
-                                         out, lse, ws, dev_err, mode == CSA2_MODE_REUSE,
-                                         reinterpret_cast<cudaStream_t>(stream)));
+                                         out, lse, ws, dev_err,
+                                         mode == CSA2_MODE_REUSE && csa2::last_call_was_attend(
+                                             reinterpret_cast<cudaStream_t>(stream)),
+                                         reinterpret_cast<cudaStream_t>(stream));
+  csa2::note_call(reinterpret_cast<cudaStream_t>(stream), true);
+  return cuda_status(launch_err);
 }
 
 int csa2_attend_queries(const void* q, float softmax_scale, const uint8_t* codes,
@@ -262,11 +289,13 @@ int csa2_attend_queries(const void* q, float softmax_scale, const uint8_t* codes
   const size_t need = csa2::attend_workspace_bytes(Q, K, W);
   if (need > 0 && (ws == nullptr || !aligned16(ws) || ws_bytes < need)) return CSA2_ERR_WORKSPACE;
   // the kernels check every qseq entry against B (a bad one gives an empty query and a flag)
-  return cuda_status(csa2::launch_attend(q, softmax_scale, codes, scales, n_cap, N, idx, K,
+  const cudaError_t launch_err = csa2::launch_attend(q, softmax_scale, codes, scales, n_cap, N, idx, K,
                                          W > 0 ? swa : nullptr, W > 0 ? swa_scale : nullptr,
                                          W > 0 ? swa_len : nullptr, W, qseq,
                                          W > 0 ? swa_lo : nullptr, S, B, Q, out, lse, ws, dev_err,
-                                         false, reinterpret_cast<cudaStream_t>(stream)));
+                                         false, reinterpret_cast<cudaStream_t>(stream));
+  csa2::note_call(reinterpret_cast<cudaStream_t>(stream), true);
+  return cuda_status(launch_err);
 }
 
 int csa2_cache_restore(const uint8_t* host_codes, const uint8_t* host_scales, const void* host_ik,
@@ -282,6 +311,7 @@ int csa2_cache_restore(const uint8_t* host_codes, const uint8_t* host_scales, co
     e = copy_rows(scales, n_cap, host_scales, n_host, CSA2_D / 16, B, N, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && ik_cache != nullptr)
     e = copy_rows(ik_cache, n_cap, host_ik, n_host, CSA2_DI * 2, B, N, cudaMemcpyHostToDevice, s);
+  csa2::note_call(reinterpret_cast<cudaStream_t>(stream), false);
   return cuda_status(e);
 }
 
@@ -318,8 +348,10 @@ int csa2_swa_replay(const void* h, const void* w, int B, int Wr, int d, const in
   if (Wr == 0) return CSA2_OK;
   if (ws == nullptr || !aligned16(ws) || ws_bytes < csa2::swa_replay_workspace_bytes(B, Wr, d))
     return CSA2_ERR_WORKSPACE;
-  return cuda_status(csa2::launch_swa_replay(h, w, B, Wr, d, N, swa, swa_scale, W, ws, dev_err,
-                                             reinterpret_cast<cudaStream_t>(stream)));
+  const cudaError_t launch_err = csa2::launch_swa_replay(h, w, B, Wr, d, N, swa, swa_scale, W, ws, dev_err,
+                                             reinterpret_cast<cudaStream_t>(stream));
+  csa2::note_call(reinterpret_cast<cudaStream_t>(stream), false);
+  return cuda_status(launch_err);
 }
 
 }  // extern "C"

@@ -13,6 +13,11 @@ void profile_begin(int kernel, cudaStream_t s);  // records the start event if o
 void profile_end(int kernel, cudaStream_t s);    // records the stop event if one is set
 int device_sm_count();        // SMs of the current device (cached per device)
 
+// The library's last call on each stream: whether it was an attention (which writes only its
+// outputs and workspace). A Reuse-mode attention starts gathering before its wait only then.
+void note_call(cudaStream_t s, bool is_attend);
+bool last_call_was_attend(cudaStream_t s);
+
 // cuTensorMapEncodeTiled from the driver (looked up once through the runtime), or null.
 typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                       const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,

@@ -98,5 +98,6 @@ extern "C" int csa2_index_reindex_noalloc(const void* iq, const float* w, const 
   const cudaError_t e = csa2::launch_index_reindex(iq, w, ik_cache, N, B, n_cap, pool, L, K, topk,
                                                    scratch, dev_err,
                                                    reinterpret_cast<cudaStream_t>(stream));
+  csa2::note_call(reinterpret_cast<cudaStream_t>(stream), false);
   return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }

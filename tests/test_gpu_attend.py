@@ -178,3 +178,39 @@ def test_query_magnitudes(gpu, qmag):
     out, lse, err = run_attend(csa2.MODE_REUSE, q, scale, cache, [n_cap], idx, [W], dev)
     ref_out, ref_lse = oracle_attend(q, scale, codes, scales, idx, swa, swsc, [W])
     check_attention(out, lse, ref_out, ref_lse)
+
+
+def test_reuse_right_after_the_index_call_that_wrote_its_indices(gpu):
+    """A Reuse-mode call straight after the Reindex call that wrote its indices (on the same
+    stream) must wait for them: the library gathers early only after its own attention calls.
+    Its output equals the Full-mode call's on the same indices, bit for bit."""
+    dev = gpu
+    B, n_cap, K, W = 4, 8192, 512, 128
+    cache, codes, scales, swa, swsc = build_cache(B, n_cap, [n_cap] * B, W, [W] * B, seed=11, dev=dev)
+    g = torch.Generator().manual_seed(11)
+    ik = torch.randn(B, n_cap, 64, generator=g).to(torch.bfloat16).to(dev)
+    iq = torch.randn(B, 4, 64, generator=g).to(torch.bfloat16).to(dev)
+    w = (torch.rand(B, 4, generator=g) + 0.5).to(dev)
+    Nt = torch.full((B,), n_cap, dtype=torch.int32, device=dev)
+    pool = torch.arange(n_cap, dtype=torch.int32, device=dev)[None].repeat(B, 1)
+    q = (torch.randn(B, 16, 512, generator=g) / math.sqrt(512)).to(torch.bfloat16).to(dev)
+    swa_len = torch.full((B,), W, dtype=torch.int32, device=dev)
+    outs = []
+    for mode in (csa2.MODE_REUSE, csa2.MODE_FULL):
+        topk = torch.full((B, K), -1, dtype=torch.int32, device=dev)
+        ws_re = csa2.workspace(csa2.index_reindex_workspace_bytes(B, n_cap, K), dev)
+        ws_at = csa2.workspace(csa2.attend_workspace_bytes(B, K, W), dev)
+        out = torch.empty(B, 16, 512, device=dev)
+        lse = torch.empty(B, 16, device=dev)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        csa2.index_reindex(iq, w, ik, Nt, pool, K, topk, ws_re, err)
+        csa2.attend(mode, q, 1.0, cache.codes, cache.scales, Nt, topk, cache.swa, cache.swa_scale,
+                    swa_len, out, lse, ws_at, err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        outs.append((out.cpu().numpy(), lse.cpu().numpy(), topk.cpu().numpy()))
+    assert np.array_equal(outs[0][2], outs[1][2])
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+    ref_out, ref_lse = oracle_attend(q.cpu(), 1.0, codes, scales, torch.from_numpy(outs[0][2]),
+                                     swa, swsc, [W] * B)
+    check_attention(outs[0][0], outs[0][1], ref_out, ref_lse)
