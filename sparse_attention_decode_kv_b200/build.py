@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libcsa2.so")
-SOURCES = ["abi.cu", "append.cu", "attend.cu", "ced.cu", "index.cu", "noalloc.cu"]
+SOURCES = ["abi.cu", "append.cu", "attend.cu", "attend_tc.cu", "ced.cu", "index.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "internal.h", "select.cuh", "swa_codec.cuh", "tcgen05.cuh"]
 
 NVCC_FLAGS = [

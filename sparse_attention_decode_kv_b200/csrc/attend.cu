@@ -538,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 // Log-sum-exp merge of the split partials: grid = (16 heads, B), 128 threads x 4 dims. Every
 // thread requests the partial (m, l) it owns and its float4 of every split's partial o at once
 // (one memory round trip), then the weights exp(m_s - m) / l are formed in shared memory.
-constexpr int kMaxSplits = 128;
+constexpr int kMaxSplits = kAttendMaxSplits;
 constexpr int kMergeBatch = 16;  // partial-o requests in flight per thread
 __global__ void __launch_bounds__(128)
     attend_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
@@ -618,10 +618,14 @@ int attend_split_count(int B, int K, int W) {
   return splits;
 }
 
+// Enough for either kernel: the tensor-core kernel falls back to this one when its operands cannot
+// be described by TMA tensor maps.
 size_t attend_workspace_bytes(int B, int K, int W) {
   const int splits = attend_split_count(B, K, W);
-  if (splits == 1) return 0;
-  return static_cast<size_t>(B) * splits * HQ * (D + 2) * sizeof(float);
+  const size_t own = splits == 1 ? 0 : static_cast<size_t>(B) * splits * HQ * (D + 2) * sizeof(float);
+  if (!attend_tc_selected(B, K, W)) return own;
+  const size_t tc = attend_tc_workspace_bytes(B, K, W);
+  return tc > own ? tc : own;
 }
 
 cudaError_t launch_attend(const void* q, float softmax_scale, const uint8_t* codes,
@@ -630,6 +634,12 @@ cudaError_t launch_attend(const void* q, float softmax_scale, const uint8_t* cod
                           const int32_t* swa_len, int W, const int32_t* qseq,
                           const int32_t* swa_lo, int S, int nseq, int B, float* out, float* lse,
                           void* ws, int32_t* dev_err, bool early_rows, cudaStream_t s) {
+  if (attend_tc_selected(B, K, W)) {
+    const cudaError_t e = launch_attend_tc(q, softmax_scale, codes, scales, n_cap, N, idx, K, swa,
+                                           swa_scale, swa_len, W, qseq, swa_lo, S, nseq, B, out, lse,
+                                           ws, dev_err, early_rows, s);
+    if (e != cudaErrorNotSupported) return e;  // else: operands TMA cannot describe
+  }
   const int splits = attend_split_count(B, K, W);
   float* part_o = nullptr;
   float* part_ml = nullptr;
@@ -663,6 +673,15 @@ cudaError_t launch_attend(const void* q, float softmax_scale, const uint8_t* cod
     if (e == cudaSuccess) e = cudaGetLastError();
   }
   profile_end(CSA2_KERNEL_ATTEND, s);
+  return e;
+}
+
+cudaError_t launch_attend_merge(const float* part_o, const float* part_ml, int nsplit, int B,
+                                float* out, float* lse, cudaStream_t s) {
+  cudaError_t e = launch_pdl(attend_merge_kernel, dim3(HQ, B), dim3(128), 0, s, part_o, part_ml,
+                             nsplit, out, lse);
+  count_launches(1);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e;
 }
 

@@ -41,6 +41,24 @@ cudaError_t launch_attend(const void* q, float softmax_scale, const uint8_t* cod
                           const int32_t* swa_lo, int S, int nseq, int B, float* out, float* lse,
                           void* ws, int32_t* dev_err, bool early_rows, cudaStream_t s);
 
+// Log-sum-exp merge of per-split partials (m, l, unnormalised o) into out and lse; nsplit <= 128.
+constexpr int kAttendMaxSplits = 128;
+cudaError_t launch_attend_merge(const float* part_o, const float* part_ml, int nsplit, int B,
+                                float* out, float* lse, cudaStream_t s);
+
+// Sparse attention on the tcgen05 tensor cores (persistent, one CTA per SM), chosen by
+// launch_attend from this batch size up.
+constexpr int kTcMinBatch = 64;
+bool attend_tc_selected(int B, int K, int W);
+int attend_tc_split_count(int B, int K, int W);
+size_t attend_tc_workspace_bytes(int B, int K, int W);
+cudaError_t launch_attend_tc(const void* q, float softmax_scale, const uint8_t* codes,
+                             const uint8_t* scales, int n_cap, const int32_t* N, const int32_t* idx,
+                             int K, const uint8_t* swa, const float* swa_scale,
+                             const int32_t* swa_len, int W, const int32_t* qseq,
+                             const int32_t* swa_lo, int S, int nseq, int B, float* out, float* lse,
+                             void* ws, int32_t* dev_err, bool early_rows, cudaStream_t s);
+
 // Full-mode indexer.
 size_t index_full_workspace_bytes(int B, int n_cap, int K, int P);
 cudaError_t launch_index_full(const void* iq, const float* w, const void* ik_cache,
