@@ -1060,7 +1060,7 @@ def run_queries(args, world, rank, local):
                          % (cache.codes.numel() * 1.125 / 1e6, swa.numel() * 1.0078 / 1e6),
                    "parallelism": f"dp{world} (independent sequences)"},
         "achieved_gbs": round(gbs, 1),
-        "roofline": {"kernel": "attend_kernel (multi-query)", "bound": "hbm",
+        "roofline": {"kernel": "attend_tc_kernel (tcgen05, multi-query)", "bound": "hbm",
                      "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(gbs / peak, 4), "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": byts,
@@ -1575,7 +1575,8 @@ def run_sweep(args, world, rank, local):
                        "l2": "flushed before every call (a 256 MB read outside the events)",
                        "parallelism": f"dp{world} (independent sequences)"},
             "calls_per_s": round(world * 1e3 / call_ms, 1),
-            "roofline": {"kernel": "attend_kernel + attend_merge_kernel (one csa2_attend call)",
+            "roofline": {"kernel": ("attend_tc_kernel (tcgen05)" if B >= 64 else
+                                    "attend_kernel + attend_merge_kernel (mma.sync)") + ", one csa2_attend call",
                          "bound": "hbm", "achieved": round(byts / (call_ms / 1e3) / 1e9, 1),
                          "peak": peak, "unit": "GB/s",
                          "frac": round(byts / (call_ms / 1e3) / 1e9 / peak, 4),

@@ -473,6 +473,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // -------------------------------------------------------------------------------- gather
     const int pw = warp == 0 ? 0 : 1;  // items 64 pw .. 64 pw + 63
     const int g = lane & 15;           // this lane's group of four items
+    if (lane == 0) {  // the tensor maps are kernel parameters: fetch them while the CTA starts
+      if (pw == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_codes)) : "memory");
+      } else {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_scales)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_swa)) : "memory");
+      }
+    }
     bool waited = a.early_rows == 0;
     if (waited) {
       pdl_wait();
