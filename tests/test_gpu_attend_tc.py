@@ -4,8 +4,8 @@ From 64 queries up `csa2_attend` runs the persistent tcgen05 kernel (`csrc/atten
 of 128 items, S^T = V q^T and O^T = V^T P^T accumulated in tensor memory, one CTA per SM looping
 over (query, split) units. These cases drive its paths: splits with partial outputs and the merge
 kernel, CTAs that take several units, ragged index and SWA tiles, several SWA tiles, no SWA, empty
-queries, invalid indices, and query magnitudes that move the softmax reference maxima between
-tiles (the lazy rescaling of O).
+queries, invalid indices, unknown sequences and clamped windows of the multi-query form, and query
+magnitudes that move the softmax reference maxima between tiles (the lazy rescaling of O).
 
 Method: "DeepSeek V4.1 Flash 拆解" (austincafe.tech), section 一 -- a Reuse layer runs sparse
 attention directly over reused indices; the main KV is MXFP4, the SWA KV FP8, both in one
@@ -33,12 +33,12 @@ def sorted_indices(rng, B, K, N, pad):
     return idx
 
 
-# (B, n_cap, K, W):
-#   64 x (512 + 128): 5 tiles, 3 splits, 192 units on 148 CTAs (some CTAs take two units)
-#   64 x (300 + 200): ragged last index tile, two SWA tiles (128 + 72 rows)
+# (B, n_cap, K, W), 148 SMs:
+#   64 x (512 + 128): 5 tiles, 2 splits per query (2 + 3 tiles), partials merged
+#   64 x (300 + 200): ragged last index tile, two SWA tiles (128 + 72 rows), 2 splits
 #   96 x 130, no SWA: two index tiles, the second with 2 items
 #   80 x (40 + 256): one short index tile, two full SWA tiles
-#   200 x (256 + 64): one split, CTAs looping over two queries
+#   200 x (256 + 64): one unit per query, 200 units on 148 CTAs (some CTAs take two)
 @pytest.mark.parametrize("B,n_cap,K,W", [(64, 1024, 512, 128), (64, 2048, 300, 200),
                                          (96, 512, 130, 0), (80, 256, 40, 256),
                                          (200, 512, 256, 64)])
@@ -155,3 +155,38 @@ def test_tc_reuse_equals_full_bit_for_bit(gpu):
             for m in (csa2.MODE_FULL, csa2.MODE_REUSE, csa2.MODE_REUSE)]
     for o, l, _ in outs[1:]:
         assert np.array_equal(o, outs[0][0]) and np.array_equal(l, outs[0][1])
+
+
+def test_tc_queries_bad_sequences_and_clamped_windows(gpu):
+    """csa2_attend_queries with 80 queries (the tcgen05 kernel): queries naming no sequence give
+    zeros and lse = -inf and are flagged; windows running past the SWA buffer are clamped and
+    flagged. Two SWA tiles per query (W = 200) start at arbitrary rows, so the tiled window loads
+    begin at odd offsets and run past the buffer's end."""
+    from test_gpu_attend_queries import _oracle_query, _run_queries, _swa_buffer
+    dev = gpu
+    B, n_cap, K, W, S = 3, 1024, 100, 200, 256
+    N = [1024, 900, 1000]
+    cache, codes, scales, _, _ = build_cache(B, n_cap, N, 0, [0] * B, seed=71, dev=dev)
+    swa, swsc = _swa_buffer(B, S, seed=72)
+    Q = 80
+    rng = np.random.default_rng(73)
+    qseq = [[0, 1, 2, -1, 5][i % 5] for i in range(Q)]
+    idx = np.full((Q, K), -1, np.int32)
+    for i in range(Q):
+        nb = N[qseq[i]] if 0 <= qseq[i] < B else 1024
+        take = K - (i % 3) * 11
+        idx[i, :take] = np.sort(rng.choice(nb, take, replace=False))
+    lo = [(37 * i) % S for i in range(Q)]
+    ln = [[200, 0, 131, 64, 199][i % 5] for i in range(Q)]
+    q = (torch.randn(Q, 16, 512, generator=torch.Generator().manual_seed(74)) /
+         math.sqrt(512)).to(torch.bfloat16)
+    out, lse, err = _run_queries(q, cache, N, qseq, idx, swa, swsc, lo, ln, W, dev)
+    assert err & csa2.DEVERR_INDEX_RANGE and err & csa2.DEVERR_NLEN
+    for i in range(Q):
+        b = qseq[i]
+        if not 0 <= b < B:
+            assert np.all(out[i] == 0) and np.all(np.isneginf(lse[i]))
+            continue
+        l = min(ln[i], S - lo[i])
+        ro, rl = _oracle_query(q[i], codes, scales, b, idx[i], swa, swsc, lo[i], l)
+        check_attention(out[i], lse[i], ro, rl)
