@@ -2,7 +2,8 @@
 // csrc/attend_tc.cu: bandwidth of random-row gathers of 256-byte code rows and 32-byte scale rows
 // (an MXFP4 cache) into shared memory, by method and by the number of issuing warps: cp.async
 // 16 B (16 lanes per row), TMA tile::gather4 (two 128-byte code halves with 128-byte swizzle plus the
-// scale rows), one cp.async.bulk per row, and plain 16-byte loads into registers. One CTA per SM,
+// scale rows), one cp.async.bulk per row, plain 16-byte loads into registers (16 lanes per row), and
+// one thread per row loading its own row (uncoalesced). One CTA per SM,
 // persistent over tiles of 128 rows, a two-slot ring and a consumer warp that touches each row.
 // All waits are bounded; every index stays inside its buffer.
 //
@@ -50,7 +51,8 @@ struct Smem {
 };
 
 // method: 0 cp.async (16 lanes per row), 1 TMA gather4 (code halves 128 B swizzled + scales),
-//         2 cp.async.bulk per row (256 B + 32 B), 3 ld.global.nc.v4 into registers (no smem)
+//         2 cp.async.bulk per row (256 B + 32 B), 3 ld.global.nc.v4 into registers (no smem),
+//         4 one thread per row, 16-byte loads of its own row into registers (no smem)
 template <int METHOD, int PW>
 __global__ void __launch_bounds__(32 * (PW + 1), 1)
     gather_kernel(const __grid_constant__ CUtensorMap mc, const __grid_constant__ CUtensorMap ms,
@@ -69,6 +71,26 @@ __global__ void __launch_bounds__(32 * (PW + 1), 1)
   __syncthreads();
   const int* my_idx = idx + (size_t)blockIdx.x * tiles_per_cta * kT;
   unsigned acc = 0;
+  if (METHOD == 4) {
+    // one thread per row: each thread loads its own row's 16 code pieces and 2 scale pieces, one
+    // tile of 128 rows per 4 warps, the next tile's pieces requested before the current are used
+    {
+      for (int e = threadIdx.x; e < tiles_per_cta * kT; e += blockDim.x) {
+        const int row = my_idx[e];
+        const uint4* src = reinterpret_cast<const uint4*>(codes + (size_t)row * 256);
+        uint4 v[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) v[c] = __ldg(src + c);
+        const uint4 s0 = __ldg(reinterpret_cast<const uint4*>(scales + (size_t)row * 32));
+        const uint4 s1 = __ldg(reinterpret_cast<const uint4*>(scales + (size_t)row * 32) + 1);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) acc ^= v[c].x ^ v[c].w;
+        acc ^= s0.y ^ s1.z;
+      }
+    }
+    sink[blockIdx.x * blockDim.x + tid] = acc;
+    return;
+  }
   if (METHOD == 3) {
     // every warp loads its share of rows straight into registers, 16 lanes per row
     const int nw = PW + 1;
@@ -208,7 +230,6 @@ int main() {
     printf("encode %d %d\n", (int)r, (int)r2);
     if (r || r2) return 1;
   }
-  run<0, 1>("cp.async 16B", mc, ms, codes, scales, idx, tiles_per_cta, sink, err, sms);
   run<0, 2>("cp.async 16B", mc, ms, codes, scales, idx, tiles_per_cta, sink, err, sms);
   run<0, 4>("cp.async 16B", mc, ms, codes, scales, idx, tiles_per_cta, sink, err, sms);
   run<0, 8>("cp.async 16B", mc, ms, codes, scales, idx, tiles_per_cta, sink, err, sms);
@@ -218,6 +239,9 @@ int main() {
   run<1, 4>("TMA gather4 (2x128B + 32B)", mc, ms, codes, scales, idx, tiles_per_cta, sink, err, sms);
   run<2, 1>("bulk per row (256B + 32B)", mc, ms, codes, scales, idx, tiles_per_cta, sink, err, sms);
   run<2, 4>("bulk per row (256B + 32B)", mc, ms, codes, scales, idx, tiles_per_cta, sink, err, sms);
+  run<4, 3>("thread per row, 16-B loads", mc, ms, codes, scales, idx, tiles_per_cta, sink, err, sms);
+  run<4, 7>("thread per row, 16-B loads", mc, ms, codes, scales, idx, tiles_per_cta, sink, err, sms);
+  run<4, 15>("thread per row, 16-B loads", mc, ms, codes, scales, idx, tiles_per_cta, sink, err, sms);
   run<3, 7>("ld.global.v4 to registers", mc, ms, codes, scales, idx, tiles_per_cta, sink, err, sms);
   run<3, 15>("ld.global.v4 to registers", mc, ms, codes, scales, idx, tiles_per_cta, sink, err, sms);
   run<3, 31>("ld.global.v4 to registers", mc, ms, codes, scales, idx, tiles_per_cta, sink, err, sms);
