@@ -816,7 +816,9 @@ CED_SHAPE = dict(B=8, n=4096, d=4096)   # 32,768 new tokens, hidden size 4,096
 
 
 def ced_cpu_baseline(h, w, rows=4096):
-    """The oracle's projection and quantisation of a few rows, scaled to TFLOP/s."""
+    """The oracle's projection and quantisation of a few rows, split over the host threads (ctypes
+    releases the GIL while the oracle runs), scaled to TFLOP/s."""
+    import concurrent.futures as cf
     import numpy as np
     import oracle
     from oracle import build as oracle_build
@@ -824,13 +826,21 @@ def ced_cpu_baseline(h, w, rows=4096):
     d = h.shape[-1]
     hb = h.reshape(-1, d)[:rows].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
     wb = w.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
-    t = time.perf_counter()
-    c, _ = oracle.ced_project(hb, wb)
-    oracle.mxfp4_quantize_f32(c.astype(np.float32))
-    sec = time.perf_counter() - t
+    threads = max(1, min(host_threads(), rows // 16, 64))
+    parts = np.array_split(hb, threads)
+
+    def one(part):
+        c, _ = oracle.ced_project(np.ascontiguousarray(part), wb)
+        oracle.mxfp4_quantize_f32(c.astype(np.float32))
+
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        t = time.perf_counter()
+        list(ex.map(one, parts))
+        sec = time.perf_counter() - t
     value = 2.0 * rows * 512 * d / sec / 1e12
-    return {"value": round(value, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-            "sample": f"{rows} token rows of d = {d} projected and quantised ({sec:.2f} s)",
+    return {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows} token rows of d = {d} projected and quantised, split over {threads} "
+                      f"threads ({sec:.2f} s)",
             "seconds": round(sec, 2)}
 
 
@@ -935,22 +945,31 @@ QUERIES_SHAPE = dict(B=8, N=131072, T=512, K=512, W=128)
 
 
 def queries_cpu_baseline(q, codes, scales, idx, swa, swsc, qseq, lo, ln, n_sample=320):
-    """The oracle's attention of a sample of the queries, scaled to queries/s."""
+    """The oracle's attention of a sample of the queries, split over the host threads (ctypes
+    releases the GIL while the oracle runs), scaled to queries/s."""
+    import concurrent.futures as cf
     import numpy as np
     import oracle
     from oracle import build as oracle_build
     oracle_build.build()
     Q = q.shape[0]
+    threads = max(1, min(host_threads(), 64))
+    n_sample = min(Q, max(n_sample, 8 * threads))
     pick = np.linspace(0, Q - 1, n_sample).astype(np.int64)
     qb = q[pick].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
-    t0 = time.perf_counter()
-    for j, i in enumerate(pick):
+
+    def one(j):
+        i = pick[j]
         b, a, n = int(qseq[i]), int(lo[i]), int(ln[i])
         oracle.attend_seq(qb[j], 1.0, codes[b], scales[b], idx[i].astype(np.int64),
                           swa[b, a:a + n], swsc[b, a:a + n], n)
-    sec = time.perf_counter() - t0
-    return {"value": round(n_sample / sec, 3), "unit": "queries/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n_sample} of {Q} queries, evenly spaced ({sec:.2f} s)",
+
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        t0 = time.perf_counter()
+        list(ex.map(one, range(n_sample)))
+        sec = time.perf_counter() - t0
+    return {"value": round(n_sample / sec, 3), "unit": "queries/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n_sample} of {Q} queries, evenly spaced, over {threads} threads ({sec:.2f} s)",
             "seconds": round(sec, 2)}
 
 
@@ -1093,22 +1112,32 @@ def replay_cpu_baseline(hc, hs, hi, hwin, w, N):
     import oracle
     from oracle import build as oracle_build
     oracle_build.build()
+    import concurrent.futures as cf
     B, W = hwin.shape[0], hwin.shape[1]
-    hb = hwin[:1].contiguous().view(torch.int16).numpy().view(np.uint16)
+    hb = hwin.contiguous().view(torch.int16).numpy().view(np.uint16)
     wb = w.contiguous().view(torch.int16).numpy().view(np.uint16)
     t0 = time.perf_counter()
     for src in (hc, hs, hi.view(torch.int16)):
         np.copy(src.numpy())
     t_copy = time.perf_counter() - t0
-    swa = np.zeros((1, W, 512), np.uint8)
-    sc = np.zeros((1, W), np.float32)
-    t0 = time.perf_counter()
-    oracle.swa_replay(hb, wb, [N], swa, sc)
-    t_rep = time.perf_counter() - t0
-    sec = t_copy + B * t_rep
-    return {"value": round(1.0 / sec, 4), "unit": "restores/s", "cores": 1, "kind": "oracle",
+    # the windows' replays, one sequence per host thread (ctypes releases the GIL)
+    threads = max(1, min(host_threads(), B))
+
+    def one(b):
+        swa = np.zeros((1, W, 512), np.uint8)
+        sc = np.zeros((1, W), np.float32)
+        oracle.swa_replay(np.ascontiguousarray(hb[b:b + 1]), wb, [N], swa, sc)
+
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        t0 = time.perf_counter()
+        list(ex.map(one, range(threads)))
+        t_rep = time.perf_counter() - t0
+    rounds = -(-B // threads)
+    sec = t_copy + rounds * t_rep
+    return {"value": round(1.0 / sec, 4), "unit": "restores/s", "cores": threads, "kind": "oracle",
             "sample": f"all {B} sequences' rows copied with numpy ({t_copy:.2f} s) + the oracle's "
-                      f"replay of 1 of {B} windows ({t_rep:.2f} s), scaled to {B}",
+                      f"replay of {threads} of {B} windows in parallel ({t_rep:.2f} s), "
+                      f"scaled to {rounds} round(s)",
             "seconds": round(t_copy + t_rep, 2)}
 
 

@@ -109,15 +109,14 @@ double oracle_e4m3_decode(uint8_t code) {
 /* Magnitudes of codes 0..126 (all non-negative finite values) in ascending order; code order is
  * magnitude order for a fixed sign. */
 static double g_e4m3_grid[127];
-static int g_e4m3_grid_ready = 0;
 
-static const double *e4m3_grid(void) {
-  if (!g_e4m3_grid_ready) {
-    for (int c = 0; c < 127; ++c) g_e4m3_grid[c] = oracle_e4m3_decode((uint8_t)c);
-    g_e4m3_grid_ready = 1;
-  }
-  return g_e4m3_grid;
+/* Filled once when the library is loaded, before any caller's thread can use it, so that
+ * concurrent callers never see a partly built table. */
+__attribute__((constructor)) static void e4m3_grid_init(void) {
+  for (int c = 0; c < 127; ++c) g_e4m3_grid[c] = oracle_e4m3_decode((uint8_t)c);
 }
+
+static const double *e4m3_grid(void) { return g_e4m3_grid; }
 
 /* Round-to-nearest-even with saturation to +-448 ("satfinite"); the sign bit is kept, so a
  * negative input that rounds to zero gives 0x80. NaN in -> 0x7F. */
