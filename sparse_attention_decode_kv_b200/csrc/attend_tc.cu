@@ -19,7 +19,8 @@
 //   warps 0, 3   gather, 64 items each: index loads, then TMA copies into a two-slot ring
 //                completing on mbarriers: tile::gather4 of four items' 128-byte code halves and
 //                32-byte scale rows per instruction, tiled 128 x 64-row loads of the contiguous SWA
-//                window (the issue rate per warp bounds a gather, so two warps issue)
+//                window (the issue rate per warp bounds a gather, so two warps issue); the CTA's
+//                first tile of indices is issued by the dequantisation warps, idle until it lands
 //   warp 1       issues QK^T (and owns the tensor-memory allocation)
 //   warp 2       issues P.V
 //   warps 4-11   dequantise, one item per thread and half the dims per warp (dim half h = the P.V
@@ -414,6 +415,18 @@ __device__ void stage_q(const TcArgs& a, int b, int st, uint32_t q_smem, TcSmall
   }
 }
 
+// The CTA's first tile is gathered by the dequantisation warps, which would otherwise wait for it,
+// when it is a tile of indices (the gather warps then only post its expected bytes). Both sides
+// decide from the same values.
+__device__ __forceinline__ bool first_tile_by_dequant(int units, int nsplit, int tiles, int tiles_idx) {
+  const int unit = static_cast<int>(blockIdx.x);
+  if (unit >= units) return false;
+  const int split = unit % nsplit;
+  const int tb = static_cast<int>(static_cast<int64_t>(split) * tiles / nsplit);
+  const int te = static_cast<int>(static_cast<int64_t>(split + 1) * tiles / nsplit);
+  return tb < te && tb < tiles_idx;
+}
+
 __global__ void __launch_bounds__(kTcThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_codes,
                      const __grid_constant__ CUtensorMap tm_scales,
@@ -489,6 +502,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int gt = 0, sn = 0;
     int fills[2] = {0, 0};  // copies issued into each slot
     bool alive = true;
+    const bool first_by_dequant = first_tile_by_dequant(units, nsplit, tiles, tiles_idx);
     for (int j = 0; alive; ++j) {
       const int unit = static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x);
       if (unit >= units) break;
@@ -534,12 +548,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (lane == 0) mbar_arrive_expect_tx(&sm.raw_full[slot], kStage / 2);
           __syncwarp();
           const uint32_t grp = static_cast<uint32_t>(16 * pw + g);  // group of 4 items in the tile
-          // lanes 0..15: code bytes 0..127 and the scale rows; lanes 16..31: code bytes 128..255
-          tma_gather4(st + (lane >> 4) * kCodeHalf + 512u * grp, &tm_codes, &sm.raw_full[slot],
-                      128 * (lane >> 4), row[0], row[1], row[2], row[3]);
-          if (lane < 16)
-            tma_gather4(st + kScalesAt + 128u * grp, &tm_scales, &sm.raw_full[slot], 0, row[0], row[1],
-                        row[2], row[3]);
+          if (gt > 0 || !first_by_dequant) {
+            // lanes 0..15: code bytes 0..127 and the scale rows; lanes 16..31: code bytes 128..255
+            tma_gather4(st + (lane >> 4) * kCodeHalf + 512u * grp, &tm_codes, &sm.raw_full[slot],
+                        128 * (lane >> 4), row[0], row[1], row[2], row[3]);
+            if (lane < 16)
+              tma_gather4(st + kScalesAt + 128u * grp, &tm_scales, &sm.raw_full[slot], 0, row[0], row[1],
+                          row[2], row[3]);
+          }
           ++fills[slot];
           sn += 1;
         } else {
@@ -694,6 +710,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int q4 = warp & 3, h = (warp - 4) >> 2;
     const int i = 32 * q4 + lane;  // item of this thread
     const uint32_t t_lane = static_cast<uint32_t>(32 * q4) << 16;
+    if (first_tile_by_dequant(units, nsplit, tiles, tiles_idx)) {
+      // the CTA's first tile into raw slot 0: this warp's 32 items, 8 groups of 4; lanes 0..7 the
+      // code half h, lanes 8..15 (h = 0 only) the scale rows
+      if (!a.early_rows) pdl_wait();
+      const int unit = static_cast<int>(blockIdx.x);
+      const int b0 = unit / nsplit, split0 = unit - b0 * nsplit;
+      const int tile0 = static_cast<int>(static_cast<int64_t>(split0) * tiles / nsplit);
+      if (lane < (h == 0 ? 16 : 8)) {
+        const QueryRows qr = query_rows(b0, a.N, a.n_cap, a.W, a.swa_len, a.qseq, a.swa_lo, a.S, a.nseq,
+                                        a.dev_err, false);
+        const int g = lane & 7;
+        const int count = min(kT, a.K - tile0 * kT);
+        int row[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int item = 32 * q4 + 4 * g + k;
+          const int p = item < count ? __ldg(a.idx + static_cast<int64_t>(b0) * a.K + tile0 * kT + item) : -1;
+          row[k] = static_cast<int>(qr.row0 + ((p >= 0 && p < qr.nb) ? p : 0));
+        }
+        const uint32_t grp = static_cast<uint32_t>(8 * q4 + g);
+        if (lane < 8)
+          tma_gather4(raw0 + static_cast<uint32_t>(h) * kCodeHalf + 512u * grp, &tm_codes, &sm.raw_full[0],
+                      128 * h, row[0], row[1], row[2], row[3]);
+        else
+          tma_gather4(raw0 + kScalesAt + 128u * grp, &tm_scales, &sm.raw_full[0], 0, row[0], row[1], row[2],
+                      row[3]);
+      }
+      __syncwarp();
+    }
     int gt = 0, sn = 0;
     bool alive = true;
     for (int j = 0; alive; ++j) {
