@@ -99,6 +99,7 @@ struct TcSmall {
   float meta_smax[3][2];       // largest valid SWA token scale of each gather warp's items (0 if none)
   float red[2][4][HQ + 1];     // per-warp tile maxima and SWA scale maximum, by tile parity
   float lred[4][HQ];           // per-warp sums of l in the epilogue
+  float scout[HQ];             // per head: the epilogue's scale of O
   float q_unscale[HQ];         // 2^(e_h - 14) * softmax_scale * log2(e)
   uint32_t tmem_base;
   int abort;
@@ -855,6 +856,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         l_part[hh] = 0.0f;
       }
       float pf_cur = 1.0f;
+      {  // the next unit's q into L2 now: it is staged from there when this unit ends
+        const int nxt = unit + static_cast<int>(gridDim.x);
+        if (nxt < units) {
+          const char* qn = reinterpret_cast<const char*>(a.q + static_cast<int64_t>(nxt / nsplit) * HQ * D);
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(qn + 128 * st) : "memory");
+        }
+      }
       for (int tile = tb; tile < te; ++tile, ++gt) {
         const bool is_swa = tile >= tiles_idx, first = tile == tb;
         const int ms = gt % 3, ss = gt & 1;
@@ -980,21 +988,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.q_full);
       }
-      float l_tot[HQ];
+      const bool single = nsplit == 1;
+      const int64_t pidx = static_cast<int64_t>(b) * nsplit + split;
+      // one head per thread (st < 16): the scale of O and lse (or m, l), while the last P.V drains
+      if (st < HQ) {
+        const float l = (sm.lred[0][st] + sm.lred[1][st]) + (sm.lred[2][st] + sm.lred[3][st]);
+        float m = -INFINITY;
 #pragma unroll
-      for (int hh = 0; hh < HQ; ++hh) l_tot[hh] = (sm.lred[0][hh] + sm.lred[1][hh]) + (sm.lred[2][hh] + sm.lred[3][hh]);
+        for (int hh = 0; hh < HQ; ++hh)
+          if (hh == st) m = m_ref[hh];
+        sm.scout[st] = single ? (l > 0.0f ? 1.0f / (l * pf_cur) : 0.0f) : 1.0f / pf_cur;
+        if (single) {
+          if (a.lse != nullptr) a.lse[static_cast<int64_t>(b) * HQ + st] = l > 0.0f ? m * kLn2 + logf(l) : -INFINITY;
+        } else {
+          a.part_ml[(pidx * HQ + st) * 2] = m == -INFINITY ? -INFINITY : m * kLn2;
+          a.part_ml[(pidx * HQ + st) * 2 + 1] = l;
+        }
+      }
+      softmax_sync();  // the scales are complete
       const bool ok = tc_wait(&sm.o_full[u & 1], static_cast<uint32_t>((u >> 1) & 1), abort);
       if (!softmax_all(ok)) {
         alive = false;
         break;
       }
       tcgen05_fence_after();
-      const bool single = nsplit == 1;
-      const int64_t pidx = static_cast<int64_t>(b) * nsplit + split;
       float sc_out[HQ];
 #pragma unroll
-      for (int hh = 0; hh < HQ; ++hh)
-        sc_out[hh] = single ? (l_tot[hh] > 0.0f ? 1.0f / (l_tot[hh] * pf_cur) : 0.0f) : 1.0f / pf_cur;
+      for (int hh = 0; hh < HQ; ++hh) sc_out[hh] = sm.scout[hh];
 #pragma unroll 1
       for (int jb = 0; jb < 4; ++jb) {
         uint32_t o[16];
@@ -1010,21 +1030,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int hh = 0; hh < HQ; ++hh) dst[hh * D + dim] = __uint_as_float(o[hh]) * sc_out[hh];
       }
-      if (st < HQ) {
-        const float l = l_tot[st];
-        float m = -INFINITY;
-#pragma unroll
-        for (int hh = 0; hh < HQ; ++hh)
-          if (hh == st) m = m_ref[hh];
-        if (single) {
-          if (a.lse != nullptr) a.lse[static_cast<int64_t>(b) * HQ + st] = l > 0.0f ? m * kLn2 + logf(l) : -INFINITY;
-        } else {
-          a.part_ml[(pidx * HQ + st) * 2] = m == -INFINITY ? -INFINITY : m * kLn2;
-          a.part_ml[(pidx * HQ + st) * 2 + 1] = l;
-        }
-      }
       tcgen05_fence_before();
-      softmax_sync();  // every thread has read lred and O before they are reused
+      softmax_sync();  // every thread has read lred, the scales and O before they are reused
       if (lane == 0) mbar_arrive(&sm.o_empty[u & 1]);
     }
     if (!alive) tc_give_up(abort, a.dev_err);
