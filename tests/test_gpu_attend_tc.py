@@ -4,8 +4,10 @@ From 64 queries up `csa2_attend` runs the persistent tcgen05 kernel (`csrc/atten
 of 128 items, S^T = V q^T and O^T = V^T P^T accumulated in tensor memory, one CTA per SM looping
 over (query, split) units. These cases drive its paths: splits with partial outputs and the merge
 kernel, CTAs that take several units, ragged index and SWA tiles, several SWA tiles, no SWA, empty
-queries, invalid indices, unknown sequences and clamped windows of the multi-query form, and query
-magnitudes that move the softmax reference maxima between tiles (the lazy rescaling of O).
+queries, invalid indices, unknown sequences and clamped windows of the multi-query form, query
+magnitudes that move the softmax reference maxima between tiles (the lazy rescaling of O), CTAs
+whose first tile is an index tile (issued by the dequantisation warps) or an SWA tile (issued by
+the gather warps), and lse requested or not on both the single-unit and the split path.
 
 Method: "DeepSeek V4.1 Flash 拆解" (austincafe.tech), section 一 -- a Reuse layer runs sparse
 attention directly over reused indices; the main KV is MXFP4, the SWA KV FP8, both in one
@@ -39,9 +41,11 @@ def sorted_indices(rng, B, K, N, pad):
 #   96 x 130, no SWA: two index tiles, the second with 2 items
 #   80 x (40 + 256): one short index tile, two full SWA tiles
 #   200 x (256 + 64): one unit per query, 200 units on 148 CTAs (some CTAs take two)
+#   64 x (40 + 256): three tiles in two splits, so every second CTA starts on an SWA tile (its
+#   first tile then comes from the gather warps, not the dequantisation warps)
 @pytest.mark.parametrize("B,n_cap,K,W", [(64, 1024, 512, 128), (64, 2048, 300, 200),
                                          (96, 512, 130, 0), (80, 256, 40, 256),
-                                         (200, 512, 256, 64)])
+                                         (200, 512, 256, 64), (64, 512, 40, 256)])
 def test_tc_attend_matches_oracle(gpu, B, n_cap, K, W):
     dev = gpu
     rng = np.random.default_rng(B * 7 + K)
@@ -76,6 +80,24 @@ def test_tc_partials_without_lse(gpu):
     idx = torch.from_numpy(sorted_indices(rng, B, K, N, [0] * B))
     q = (torch.randn(B, 16, 512, generator=torch.Generator().manual_seed(22)) * 0.05).to(torch.bfloat16)
     out, lse, err = run_attend(csa2.MODE_FULL, q, 1.0, cache, N, idx, swa_len, dev, with_lse=False)
+    assert err == 0 and lse is None
+    ref_out, _ = oracle_attend(q, 1.0, codes, scales, idx, swa, swsc, swa_len)
+    check_attention(out, None, ref_out, None)
+
+
+def test_tc_single_split_without_lse(gpu):
+    """One unit per query (no partials) with lse not requested: the epilogue writes out only."""
+    dev = gpu
+    B, n_cap, K, W = 96, 1024, 384, 128
+    assert csa2.attend_workspace_bytes(B, K, W) >= 0
+    N = [n_cap - 16 * (b % 3) for b in range(B)]
+    swa_len = [W - (b % 5) for b in range(B)]
+    cache, codes, scales, swa, swsc = build_cache(B, n_cap, N, W, swa_len, seed=23, dev=dev)
+    rng = np.random.default_rng(23)
+    idx = torch.from_numpy(sorted_indices(rng, B, K, N, [(b % 3) * 5 for b in range(B)]))
+    q = (torch.randn(B, 16, 512, generator=torch.Generator().manual_seed(24)) /
+         math.sqrt(512)).to(torch.bfloat16)
+    out, lse, err = run_attend(csa2.MODE_REUSE, q, 1.0, cache, N, idx, swa_len, dev, with_lse=False)
     assert err == 0 and lse is None
     ref_out, _ = oracle_attend(q, 1.0, codes, scales, idx, swa, swsc, swa_len)
     check_attention(out, None, ref_out, None)
